@@ -1,0 +1,88 @@
+"""Plants plausible mistakes in the oracle (on the CPU) and checks that at
+least one of its pins fails for each, so the pins are not vacuous."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+import tests.test_oracle_pins as P
+
+_orig_rows = O.attention_rows
+_orig_merge = O.merge
+
+
+def _rows_natural_log(q, k, v, scale):
+    o, l = _orig_rows(q, k, v, scale)
+    return o, l * math.log(2.0)                    # LSE left in natural units
+
+
+def _rows_no_scale(q, k, v, scale):
+    return _orig_rows(q, k, v, 1.0)
+
+
+def _rows_scale_twice(q, k, v, scale):
+    return _orig_rows(q, k, v, scale * scale)
+
+
+def _rows_transposed_v(q, k, v, scale):
+    o, l = _orig_rows(q, k, v, scale)
+    return o[:, ::-1].copy(), l                    # channel order reversed
+
+
+def _rows_drop_last_key(q, k, v, scale):
+    if k.shape[0] > 1:
+        return _orig_rows(q, k[:-1], v[:-1], scale)
+    return _orig_rows(q, k, v, scale)
+
+
+def _merge_natural(o_parts, lse_parts):
+    op, lp = O.to_f64(o_parts), O.to_f64(lse_parts)
+    M = lp.max(axis=0)
+    w = np.exp(lp - M[None])                       # e instead of 2
+    W = w.sum(axis=0)
+    return (w[..., None] * op).sum(0) / W[..., None], M + np.log2(W)
+
+
+def _shift_wrong_sign(q_rows, mu, scale):
+    return -scale * (np.asarray(q_rows) @ np.asarray(mu)) / math.log(2.0)
+
+
+PIN_TESTS = [
+    lambda g: [P.test_brute_force_tiny(s) for s in range(6)],
+    lambda g: [P.test_against_torch_float64(s) for s in range(3)],
+    lambda g: P.test_closed_forms(),
+    lambda g: P.test_randn_lse_near_log2_kv_len(g),
+    lambda g: P.test_per16_store_error_magnitude(g),
+    lambda g: P.test_smooth_k_invariance(),
+    lambda g: [P.test_merge_of_splits_equals_full(s) for s in range(4)],
+    lambda g: P.test_merge_special_cases(),
+    lambda g: P.test_chunked_merge_equals_full_with_smoothing(),
+]
+
+
+def _some_pin_fails(golden_dir):
+    for t in PIN_TESTS:
+        try:
+            t(golden_dir)
+        except (AssertionError, ValueError, IndexError):
+            return True
+    return False
+
+
+@pytest.mark.parametrize("name,attr,fn", [
+    ("natural log", "attention_rows", _rows_natural_log),
+    ("scale dropped", "attention_rows", _rows_no_scale),
+    ("scale squared", "attention_rows", _rows_scale_twice),
+    ("value channels permuted", "attention_rows", _rows_transposed_v),
+    ("last key dropped", "attention_rows", _rows_drop_last_key),
+    ("merge weights in base e", "merge", _merge_natural),
+    ("smoothing shift sign", "smooth_shift", _shift_wrong_sign),
+])
+def test_planted_mistake_is_caught(monkeypatch, golden_dir, name, attr, fn):
+    monkeypatch.setattr(O, attr, fn)
+    assert _some_pin_fails(golden_dir), f"no pin caught: {name}"
+
+
+def test_unmutated_oracle_passes_all(golden_dir):
+    assert not _some_pin_fails(golden_dir)

@@ -1,0 +1,447 @@
+"""Pins of the FP64 oracle to what the pages and the mathematics fix.
+
+None of these tests retypes the oracle's formula: each checks it against a
+brute-force enumeration, a library routine (torch float64 logsumexp/softmax),
+a closed form, an invariant, or a number the pages print.  Each is chosen so
+that a plausible slip in the oracle (natural log instead of log2, scale
+dropped or applied twice, a transposed operand, a wrong GQA head, an
+off-by-one range, a sign error in the smoothing shift) fails at least one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+
+LN2 = math.log(2.0)
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- definition
+
+@pytest.mark.parametrize("seed", range(6))
+def test_brute_force_tiny(seed):
+    """Hand enumeration of sum_j exp(s_j) with plain Python floats, D<=4, Sk<=6."""
+    r = _rng(seed)
+    n, m, D = int(r.integers(1, 4)), int(r.integers(1, 7)), int(r.integers(1, 5))
+    q, k, v = r.normal(size=(n, D)), r.normal(size=(m, D)), r.normal(size=(m, D))
+    scale = float(r.uniform(0.2, 1.5))
+    o, lse = O.attention_rows(q, k, v, scale)
+    for i in range(n):
+        z = 0.0
+        num = [0.0] * D
+        for j in range(m):
+            s = 0.0
+            for d in range(D):
+                s += q[i][d] * k[j][d]
+            w = math.exp(scale * s)
+            z += w
+            for d in range(D):
+                num[d] += w * v[j][d]
+        assert abs(lse[i] - math.log(z) / LN2) < 1e-12
+        for d in range(D):
+            assert abs(o[i][d] - num[d] / z) < 1e-12
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_against_torch_float64(seed):
+    """Library routine: LSE * ln2 == torch.logsumexp(scale*QK^T), O == softmax @ V."""
+    r = _rng(100 + seed)
+    q, k, v = r.normal(size=(17, 32)), r.normal(size=(23, 32)), r.normal(size=(23, 32))
+    scale = 32 ** -0.5
+    o, lse = O.attention_rows(q, k, v, scale)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    logits = scale * tq @ tk.T
+    np.testing.assert_allclose(lse * LN2, torch.logsumexp(logits, -1).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o, (torch.softmax(logits, -1) @ tv).numpy(), rtol=0, atol=1e-12)
+
+
+def test_closed_forms():
+    r = _rng(7)
+    D, m = 8, 9
+    k, v = r.normal(size=(m, D)), r.normal(size=(m, D))
+    # q = 0: LSE = log2 |J| exactly, O = mean of v
+    o, lse = O.attention_rows(np.zeros((1, D)), k, v, 0.7)
+    assert lse[0] == pytest.approx(math.log2(m), abs=1e-13)
+    np.testing.assert_allclose(o[0], v.mean(0), atol=1e-13)
+    # one key: LSE = scale q.k / ln2, O = v
+    q = r.normal(size=(1, D))
+    o, lse = O.attention_rows(q, k[:1], v[:1], 0.3)
+    assert lse[0] == pytest.approx(0.3 * float(q[0] @ k[0]) / LN2, abs=1e-12)
+    np.testing.assert_allclose(o[0], v[0], atol=1e-13)
+    # all keys equal: LSE = log2|J| + s/ln2
+    kk = np.repeat(k[:1], m, axis=0)
+    o, lse = O.attention_rows(q, kk, v, 0.3)
+    assert lse[0] == pytest.approx(math.log2(m) + 0.3 * float(q[0] @ k[0]) / LN2, abs=1e-12)
+    # two keys: log2(e^a + e^b), with a, b far apart and of both signs
+    for a, b in ((3.0, -2.0), (150.0, 149.0), (-400.0, -401.5)):
+        qq = np.array([[1.0, 0.0]])
+        k2 = np.array([[a, 0.0], [b, 0.0]])
+        o, lse = O.attention_rows(qq, k2, np.eye(2), 1.0)
+        ref = (max(a, b) + math.log1p(math.exp(-abs(a - b)))) / LN2
+        assert lse[0] == pytest.approx(ref, abs=1e-12)
+        assert o[0, 0] == pytest.approx(1.0 / (1.0 + math.exp(b - a)), abs=1e-12)
+    # one key dominating by > 60 nats: O = v_j*, LSE = s_j*/ln2
+    q = np.zeros((1, D)); q[0, 0] = 1.0
+    kd = r.normal(size=(m, D)) * 0.1
+    kd[4, 0] = 80.0
+    o, lse = O.attention_rows(q, kd, v, 1.0)
+    np.testing.assert_allclose(o[0], v[4], atol=1e-20 + 1e-15)
+    assert lse[0] == pytest.approx(80.0 / LN2, abs=1e-12)
+
+
+def test_empty_range():
+    o, lse = O.attention_rows(np.ones((3, 4)), np.zeros((0, 4)), np.zeros((0, 4)), 1.0)
+    assert np.all(o == 0) and np.all(np.isneginf(lse))
+
+
+def test_gqa_head_mapping():
+    """Query head h reads kv head h // G: make each kv head's keys distinct and
+    check each query head against a single-head run on the intended kv head."""
+    d = W.dense_case(1, 6, 2, 5, 11, 8, seed=3, dtype="fp32")
+    o, lse = O.dense(d["q"], d["k"], d["v"], d["scale"])
+    q, k, v = (O.to_f64(d[x]) for x in "qkv")
+    for h in range(6):
+        oh, lh = O.attention_rows(q[0, h], k[0, h // 3], v[0, h // 3], d["scale"])
+        np.testing.assert_allclose(lse[0, h], lh, atol=0)
+        other = 1 - h // 3
+        _, lo = O.attention_rows(q[0, h], k[0, other], v[0, other], d["scale"])
+        assert np.abs(lo - lse[0, h]).max() > 1e-3
+
+
+def test_nhd_matches_hnd():
+    d = W.dense_case(2, 4, 2, 7, 13, 16, seed=5, dtype="bf16")
+    o1, l1 = O.dense(d["q"], d["k"], d["v"], d["scale"], "HND")
+    qn, kn, vn = (W.to_layout(d[x], "NHD") for x in "qkv")
+    o2, l2 = O.dense(qn, kn, vn, d["scale"], "NHD")
+    np.testing.assert_array_equal(o1.transpose(0, 2, 1, 3), o2)
+    np.testing.assert_array_equal(l1, l2)
+    rows = [(1, 3, 6), (0, 0, 0), (1, 2, 4)]
+    orows, lrows = O.dense(d["q"], d["k"], d["v"], d["scale"], "HND", rows=rows)
+    for r, (b, h, i) in enumerate(rows):
+        np.testing.assert_allclose(orows[r], o1[b, h, i], atol=1e-14)
+        assert lrows[r] == pytest.approx(l1[b, h, i], abs=1e-13)
+
+
+# -------------------------------------------------- the ARK issue's numbers
+
+def test_randn_lse_near_log2_kv_len(golden_dir):
+    """k ~ N(0, I): s_j ~ N(0, sigma_i^2) with sigma_i = scale*|q_i|, so
+    LSE_i ~= log2(Sk) + sigma_i^2 / (2 ln 2) while sigma_i^2 << 2 ln Sk.  The
+    issue: with randn inputs every row's LSE is about log2(kv_len)."""
+    d = W.config1("rows")
+    _, lse = O.dense(d["q"], d["k"], d["v"], d["scale"])
+    q = O.to_f64(d["q"])
+    sig = d["scale"] * np.linalg.norm(q, axis=-1)
+    pred = math.log2(1000) + sig ** 2 / (2 * LN2)
+    mask = sig <= 1.5
+    assert mask.sum() > 60
+    assert np.abs(pred - lse)[mask].max() < 0.35
+    # printed reference rows 12..19 (another RNG stream): same magnitudes
+    g = json.load(open(os.path.join(golden_dir, "ark_issue_repro.json")))
+    ref = np.array(g["reference_lse_log2_rows_12_to_19"])
+    assert np.abs(lse[0, 0, 12:20] - ref).max() < 0.5
+
+
+def test_row_distinctness_and_blocks():
+    d = W.config1("rows")
+    _, lse = O.dense(d["q"], d["k"], d["v"], d["scale"])
+    # rows scaled by distinct factors: no two rows of a head share an LSE, and
+    # every 16-row block spans a wide range (what a per-16 store would flatten)
+    for h in range(4):
+        diffs = np.abs(lse[0, h][:, None] - lse[0, h][None, :])[np.triu_indices(64, 1)]
+        assert diffs.min() > 1e-6
+    spread = lse.reshape(4, 4, 16).max(-1) - lse.reshape(4, 4, 16).min(-1)
+    assert spread.min() > 0.1
+    db = W.config1("blocks")
+    _, lb = O.dense(db["q"], db["k"], db["v"], db["scale"])
+    blocks = lb.reshape(1, 4, 4, 16)
+    assert np.all(blocks == blocks[..., :1])
+    # distinct blocks differ
+    assert np.all(np.abs(np.diff(blocks[..., 0], axis=-1)) > 1e-3)
+
+
+def _per16_store_bug(lse):
+    """An epilogue that stores the last row of each 16-row group to all 16 slots."""
+    B, H, S = lse.shape
+    return np.repeat(lse.reshape(B, H, S // 16, 16)[..., -1:], 16, axis=-1).reshape(B, H, S)
+
+
+def test_per16_store_error_magnitude(golden_dir):
+    """The issue prints max|lse - ref| = 9.093 for the per-16-row store on
+    rows that differ, 0.000 on 16 equal rows.  Over seeds, the oracle's
+    distribution of that error must bracket the printed value."""
+    g = json.load(open(os.path.join(golden_dir, "ark_issue_repro.json")))
+    errs = []
+    for seed in range(12):
+        d = W.config1("rows", seed=seed)
+        _, lse = O.dense(d["q"], d["k"], d["v"], d["scale"])
+        errs.append(np.abs(_per16_store_bug(lse) - lse).max())
+    errs = np.array(errs)
+    printed = g["per16_store_error_rows_differ_sdpa"]
+    assert errs.min() < printed < errs.max() * 1.05
+    assert 0.5 * printed < np.median(errs) < 2.0 * printed
+    db = W.config1("blocks")
+    _, lb = O.dense(db["q"], db["k"], db["v"], db["scale"])
+    assert np.abs(_per16_store_bug(lb) - lb).max() == g["per16_store_error_16_equal_rows_sdpa"]
+
+
+# ------------------------------------------------------------------ smooth_k
+
+def test_smooth_k_invariance():
+    """O is unchanged by subtracting mean(k); LSE' + scale*q.mean(k)/ln2 = LSE."""
+    d = W.config1("koff")
+    q, k, v = (O.to_f64(d[x])[0] for x in "qkv")
+    for h in range(4):
+        o, lse = O.attention_rows(q[h], k[h], v[h], d["scale"])
+        o2, lse_corr, lse_s = O.smoothed_attention_rows(q[h], k[h], v[h], d["scale"])
+        np.testing.assert_allclose(o2, o, atol=1e-12)
+        np.testing.assert_allclose(lse_corr, lse, atol=1e-12)
+    # closed form for the shift: adding a constant c to every key element adds
+    # c*scale*sum_d(q_d) to every logit of the row, so the LSE moves by that over
+    # ln 2, while the smoothed (uncorrected) LSE does not move at all
+    c = 0.75
+    for h in range(4):
+        _, l0 = O.attention_rows(q[h], k[h], v[h], d["scale"])
+        _, l1 = O.attention_rows(q[h], k[h] + c, v[h], d["scale"])
+        np.testing.assert_allclose(l1 - l0, c * d["scale"] * q[h].sum(-1) / LN2, atol=1e-10)
+        _, _, s0 = O.smoothed_attention_rows(q[h], k[h], v[h], d["scale"])
+        _, _, s1 = O.smoothed_attention_rows(q[h], k[h] + c, v[h], d["scale"])
+        np.testing.assert_allclose(s1, s0, atol=1e-10)
+
+
+def test_smooth_k_uncorrected_error_magnitude(golden_dir):
+    """The issue prints an uncorrected smooth_k LSE error of 3.727 (16 equal
+    rows, K + 0.5); over seeds the oracle's shift magnitude brackets it."""
+    g = json.load(open(os.path.join(golden_dir, "ark_issue_repro.json")))
+    vals = []
+    for seed in range(12):
+        d = W.config1("koff", seed=seed)
+        q, k = O.to_f64(d["q"])[0], O.to_f64(d["k"])[0]
+        vals.append(max(np.abs(O.smooth_shift(q[h], O.kv_mean(k[h]), d["scale"])).max()
+                        for h in range(4)))
+    printed = g["smooth_k_uncorrected_error_16_equal_rows_k_plus_half"]
+    assert min(vals) < printed < max(vals)
+    assert 0.5 * printed < np.median(vals) < 2.0 * printed
+
+
+# --------------------------------------------------------------------- merge
+
+@pytest.mark.parametrize("seed", range(4))
+def test_merge_of_splits_equals_full(seed):
+    r = _rng(200 + seed)
+    n, m, D = 5, int(r.integers(2, 60)), 16
+    q, k, v = r.normal(size=(n, D)) * 3, r.normal(size=(m, D)), r.normal(size=(m, D))
+    o, lse = O.attention_rows(q, k, v, 0.25)
+    cuts = sorted(set([0, m] + list(r.integers(0, m + 1, size=3))))
+    parts = [O.attention_rows(q, k[a:b], v[a:b], 0.25) for a, b in zip(cuts[:-1], cuts[1:])]
+    # include an empty part explicitly
+    parts.append(O.attention_rows(q, k[:0], v[:0], 0.25))
+    om, lm = O.merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    np.testing.assert_allclose(om, o, atol=1e-12)
+    np.testing.assert_allclose(lm, lse, atol=1e-12)
+    # permutation invariance
+    perm = r.permutation(len(parts))
+    om2, lm2 = O.merge(np.stack([parts[i][0] for i in perm]), np.stack([parts[i][1] for i in perm]))
+    np.testing.assert_allclose(om2, om, atol=1e-13)
+    np.testing.assert_allclose(lm2, lm, atol=1e-13)
+
+
+def test_merge_special_cases():
+    r = _rng(9)
+    o1, l1 = r.normal(size=(3, 4)), r.normal(size=3) * 50
+    om, lm = O.merge(o1[None], l1[None])
+    np.testing.assert_allclose(om, o1, atol=0)
+    np.testing.assert_allclose(lm, l1, atol=0)
+    om, lm = O.merge(np.stack([o1, o1]), np.stack([l1, l1]))
+    np.testing.assert_allclose(om, o1, atol=1e-14)
+    np.testing.assert_allclose(lm, l1 + 1.0, atol=1e-13)
+    junk = np.full((3, 4), 1e30)
+    om, lm = O.merge(np.stack([o1, junk]), np.stack([l1, np.full(3, -np.inf)]))
+    np.testing.assert_allclose(om, o1, atol=1e-14)
+    np.testing.assert_allclose(lm, l1, atol=1e-13)
+    om, lm = O.merge(np.stack([junk, junk]), np.full((2, 3), -np.inf))
+    assert np.all(om == 0) and np.all(np.isneginf(lm))
+    # LSEs spanning +-150 log2 units: exact weights
+    om, lm = O.merge(np.stack([o1, o1 * 2]), np.stack([np.full(3, 150.0), np.full(3, -150.0)]))
+    np.testing.assert_allclose(lm, 150.0, atol=1e-12)
+    np.testing.assert_allclose(om, o1, atol=1e-12)
+
+
+def test_chunked_merge_equals_full_with_smoothing():
+    """Ring-style: per-chunk smoothed partials, corrected, merge to the full run."""
+    d = W.dense_case(1, 2, 2, 9, 40, 8, seed=11, dtype="bf16", k_offset=0.5)
+    q, k, v = (O.to_f64(d[x])[0] for x in "qkv")
+    bounds = [0, 7, 19, 33, 40]
+    for h in range(2):
+        o, lse = O.attention_rows(q[h], k[h], v[h], d["scale"])
+        parts = [O.smoothed_attention_rows(q[h], k[h, a:b], v[h, a:b], d["scale"])
+                 for a, b in zip(bounds[:-1], bounds[1:])]
+        om, lm = O.merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+        np.testing.assert_allclose(om, o, atol=1e-12)
+        np.testing.assert_allclose(lm, lse, atol=1e-12)
+        # without the correction the chunks sit on different scales
+        om_bad, lm_bad = O.merge(np.stack([p[0] for p in parts]), np.stack([p[2] for p in parts]))
+        assert np.abs(om_bad - o).max() > 1e-4
+
+
+# ------------------------------------------------------- varlen and decode
+
+def test_varlen_equals_dense_per_sequence():
+    lens_q, lens_k = [3, 0, 17, 5], [4, 6, 0, 21]
+    d = W.varlen_case(lens_q, lens_k, 4, 2, 16, seed=4)
+    o, lse = O.varlen(d["q"], d["k"], d["v"], d["cu_seqlens_q"], d["cu_seqlens_k"], d["scale"])
+    q, k, v = (O.to_f64(d[x]) for x in "qkv")
+    cq, ck = d["cu_seqlens_q"].tolist(), d["cu_seqlens_k"].tolist()
+    for b in range(4):
+        qb = q[cq[b]:cq[b + 1]].transpose(1, 0, 2)[None]
+        kb = k[ck[b]:ck[b + 1]].transpose(1, 0, 2)[None]
+        vb = v[ck[b]:ck[b + 1]].transpose(1, 0, 2)[None]
+        ob, lb = O.dense(qb, kb, vb, d["scale"])
+        np.testing.assert_allclose(o[cq[b]:cq[b + 1]], ob[0].transpose(1, 0, 2), atol=1e-14)
+        np.testing.assert_allclose(lse[:, cq[b]:cq[b + 1]], lb[0], atol=1e-14)
+    # sequence 2 has queries but no keys: O = 0, LSE = -inf
+    assert np.all(o[cq[2]:cq[3]] == 0) and np.all(np.isneginf(lse[:, cq[2]:cq[3]]))
+
+
+def test_lse_layout_adapters():
+    """[H, T] varlen LSE of equal-length sequences equals the dense [B, H, S]
+    after reshape(H, B, S).transpose(0, 1) (SGLang PR thread); the Ascend
+    [T, H, 1] layout squeezed and transposed is the same [H, T]."""
+    B, S, H, D = 3, 5, 2, 8
+    d = W.varlen_case([S] * B, [S + 2] * B, H, H, D, seed=8)
+    _, lse_ht = O.varlen(d["q"], d["k"], d["v"], d["cu_seqlens_q"], d["cu_seqlens_k"], d["scale"])
+    q = O.to_f64(d["q"]).reshape(B, S, H, D)
+    k = O.to_f64(d["k"]).reshape(B, S + 2, H, D)
+    v = O.to_f64(d["v"]).reshape(B, S + 2, H, D)
+    _, lse_dense = O.dense(q, k, v, d["scale"], "NHD")
+    np.testing.assert_allclose(O.lse_varlen_to_dense(lse_ht, B, S), lse_dense, atol=1e-14)
+    lse_thl = lse_ht.T[..., None]                   # Ascend [T, H, 1]
+    np.testing.assert_array_equal(lse_thl.squeeze(-1).T, lse_ht)
+
+
+def test_decode_equals_dense_and_kv_len():
+    d = W.decode_case(8, 2, 16, 3, 50, B=2, seed=12)
+    o, lse = O.decode(d["q"], d["k"], d["v"], d["scale"])
+    od, ld = O.dense(d["q"], d["k"], d["v"], d["scale"])
+    np.testing.assert_array_equal(o, od)
+    np.testing.assert_array_equal(lse, ld)
+    o2, l2 = O.decode(d["q"], d["k"], d["v"], d["scale"], kv_len=[17, 0])
+    od2, ld2 = O.dense(d["q"][:1], d["k"][:1, :, :17], d["v"][:1, :, :17], d["scale"])
+    np.testing.assert_allclose(o2[:1], od2, atol=0)
+    np.testing.assert_allclose(l2[:1], ld2, atol=0)
+    assert np.all(o2[1] == 0) and np.all(np.isneginf(l2[1]))
+
+
+# ------------------------------------------------- large logits, fixed phi
+
+def _fixed_phi_fp32(q, k, v, scale, phi=5.0):
+    """The anti-pattern of the split-K PR: exp(s - phi) in fp32 with no max."""
+    s = (scale * q.float() @ k.float().transpose(-1, -2))
+    p = torch.exp(s - phi)
+    return (p @ v.float()) / p.sum(-1, keepdim=True)
+
+
+@pytest.mark.parametrize("Lq", [1, 2, 4])
+def test_fixed_phi_nan_counts_match_printed(golden_dir, Lq):
+    """All-positive logits of the D=128, H_q=32 decode shape: a fixed offset
+    yields NaN in every output element, the counts the PR review prints
+    (4096/8192/16384 for Lq=1/2/4); the oracle stays finite."""
+    g = json.load(open(os.path.join(golden_dir, "executorch_splitk.json")))
+    d = W.config2(Lq, 512, planted="allpos")
+    qf = d["q"].float()
+    kf, vf = d["k"].float().repeat_interleave(4, dim=1), d["v"].float().repeat_interleave(4, dim=1)
+    smin = float((d["scale"] * qf @ kf.transpose(-1, -2)).min())
+    assert smin > 88.8            # exp overflows fp32 for every logit
+    out = _fixed_phi_fp32(qf, kf, vf, d["scale"], g["fixed_phi"])
+    assert int(torch.isnan(out).sum()) == g["nan_count_by_Lq_fixed_phi"][str(Lq)]
+    o, lse = O.decode(d["q"], d["k"], d["v"], d["scale"])
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+
+
+def test_all_negative_logits_underflow_case():
+    d = W.config2(1, 512, planted="allneg")
+    qf = d["q"].float()
+    kf = d["k"].float().repeat_interleave(4, dim=1)
+    s = d["scale"] * qf @ kf.transpose(-1, -2)
+    assert float(s.max()) < -110
+    out = _fixed_phi_fp32(qf, kf, d["v"].float().repeat_interleave(4, dim=1), d["scale"])
+    assert not torch.isfinite(out).all()          # 0/0 once every weight underflows
+    o, lse = O.decode(d["q"], d["k"], d["v"], d["scale"])
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    # LSE equals the brute-force value computed around the row max
+    q64, k64 = O.to_f64(d["q"]), O.to_f64(d["k"])
+    s0 = d["scale"] * q64[0, 0, 0] @ k64[0, 0].T
+    ref = (s0.max() + math.log(np.exp(s0 - s0.max()).sum())) / LN2
+    assert lse[0, 0, 0] == pytest.approx(ref, abs=1e-10)
+
+
+def test_planted_keys_reach_150():
+    d = W.config2(1, 300, planted="pos")
+    q, k = O.to_f64(d["q"]), O.to_f64(d["k"])
+    s = d["scale"] * q[0, 0, 0] @ k[0, 0].T
+    assert 140 < s.max() < 160
+    o, lse = O.decode(d["q"], d["k"], d["v"], d["scale"])
+    # brute force around the max: the planted keys dominate every other term
+    ref = (s.max() + math.log(sum(math.exp(x - s.max()) for x in s))) / LN2
+    assert lse[0, 0, 0] == pytest.approx(ref, abs=1e-9)
+    n_top = int((s > s.max() - 1.0).sum())
+    assert lse[0, 0, 0] == pytest.approx(s.max() / LN2 + math.log2(n_top), abs=0.05)
+
+
+# ------------------------------------------------------- integer planning
+
+def test_split_bounds_partition():
+    """Bounds cover [0, n) exactly, in order, and the chunk is the smallest
+    multiple of 64 keys with which S splits cover n (found by search)."""
+    for n in [0, 1, 63, 64, 65, 1000, 4096, 32768, 40000]:
+        for S in [1, 2, 3, 7, 16, 37, 64]:
+            b = O.split_bounds(n, S)
+            assert len(b) == S + 1 and b[0] == 0 and b[-1] == n
+            assert all(x <= y for x, y in zip(b[:-1], b[1:]))
+            if n == 0:
+                continue
+            c = 64
+            while S * c < n:
+                c += 64
+            lens = [y - x for x, y in zip(b[:-1], b[1:])]
+            nonempty = [x for x in lens if x]
+            assert all(x == c for x in nonempty[:-1]) and 0 < nonempty[-1] <= c
+            assert lens[len(nonempty):] == [0] * (S - len(nonempty))
+
+
+def test_split_plan_hand_values():
+    # Lkv = 32768 over 8 kv heads on 148 SMs: ceil(296 / 8) = 37 splits,
+    # C = roundup(ceil(32768/37)=886, 64) = 896, ceil(32768/896) = 37
+    assert O.auto_num_splits(1, 8, 32, 1, 32768, 148) == 37
+    assert O.split_bounds(32768, 37)[1] == 896
+    assert O.split_bounds(32768, 37)[-2] == 36 * 896
+    # Lkv = 4096: 37 capped to ceil(4096/128) = 32; C = 128 -> 32 splits
+    assert O.auto_num_splits(1, 8, 32, 1, 4096, 148) == 32
+    # D256 shape (4 kv heads, G*Lq = 16): ceil(296/4) = 74, Lkv 16384 -> C = 256 -> 64
+    assert O.auto_num_splits(1, 4, 16, 4, 16384, 148) == 64
+    # G*Lq = 32 rows -> two row groups per kv head
+    assert O.auto_num_splits(1, 4, 16, 8, 16384, 148) == 37
+    assert O.auto_num_splits(1, 8, 32, 1, 0, 148) == 1
+    assert O.auto_num_splits(1, 8, 32, 1, 100, 148) == 1
+
+
+def test_varlen_schedule_config4():
+    cu = np.array([0, 512, 1536, 3584, 7680])
+    order, offsets, items = O.varlen_schedule(cu, cu, 24, 256)
+    assert order == [3, 2, 1, 0]
+    assert offsets == [0, 384, 576, 672, 720]
+    assert len(items) == 720 and items[0] == (3, 0, 0) and items[16] == (3, 1, 0)
+    assert items[-1] == (0, 23, 1)
+    # ties keep index order; empty-query sequences contribute nothing
+    order, offsets, items = O.varlen_schedule([0, 10, 10, 300, 310], [0, 5, 9, 9, 13], 2, 256)
+    assert order == [0, 1, 3, 2]
+    assert offsets == [0, 2, 2, 4, 8]
