@@ -1,0 +1,218 @@
+/*
+ * splitkv.h -- C ABI of the B200 (sm_100a) attention-with-LSE library.
+ *
+ * Three device operations and their host-side planning helpers:
+ *
+ *   attn_fwd_lse         prefill / varlen attention forward writing O and one
+ *                        log2 LSE per query row;
+ *   attn_splitkv_decode  split-KV decode for 1..4 query rows per head with a
+ *                        stable per-split online softmax, merged on device;
+ *   merge_state          combines partial (O, LSE) pairs of disjoint KV ranges.
+ *
+ * The quantity (all entry points): for query row i of head h and the KV range J
+ * of the call, s_j = scale * q_i . k_j and
+ *
+ *     LSE_i = log2( sum_{j in J} exp(s_j) ),  O_i = sum_j exp(s_j) v_j / sum_j exp(s_j)
+ *
+ * over the ORIGINAL, unsmoothed logits: natural exponentials, reported in log2
+ * units, one value per row ("ARK return_lse gives the same LSE for every 16
+ * query rows", auto-round issue #2556, "Expected:" in Problem Description).
+ * An empty KV range gives O_i = 0 and LSE_i = -inf.
+ *
+ * Conventions (SGLang PR #33840 "[XPU] Support softmax_lse in sgl_kernel::fwd
+ * API", Modifications and the review thread):
+ *   - outputs are written in place into caller-owned device buffers; the return
+ *     value is only a status;
+ *   - the LSE output is optional: a NULL lse pointer means "do not store it";
+ *   - the varlen (packed TND) path writes a 2-D LSE [H, total_q]; the dense
+ *     paths write a 3-D LSE [B, H, S_q].
+ * Shapes that do not satisfy the contract are rejected with a status, never
+ * reshaped silently (SGLang Ascend backend record "Unexpected Ascend TND
+ * softmax LSE shape").  There is no fixed exponent offset ("phi"): the split
+ * path uses a per-split running max (ExecuTorch PR #22133 "Prevent Voxtral
+ * NaNs in CUDA split-K attention").
+ *
+ * Memory and ownership: every pointer named "device" must point to device
+ * memory of the current CUDA device; the library never allocates device memory
+ * and keeps no per-call state.  Scratch space is the caller's "workspace",
+ * sized by the matching *_workspace() query.  All device entry points are
+ * asynchronous on `stream` (NULL = the legacy default stream), validate every
+ * argument on the host first and launch nothing if validation fails.
+ *
+ * Element types: bf16 or fp16 for q/k/v/out (q, k, v and out share one type);
+ * LSE is always fp32.  Head dimension D in {64, 128, 256} (prefill: {64, 128}).
+ * Pointers passed as tensors must be 16-byte aligned.
+ *
+ * Thread safety: entry points may be called from several host threads; calls
+ * that share a workspace must not overlap on the device.
+ */
+#ifndef SPLITKV_H_
+#define SPLITKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* skv_stream_t;
+
+typedef enum {
+  SKV_OK = 0,
+  SKV_ERR_INVALID_ARG = 1,        /* a size, pointer, alignment or layout is invalid */
+  SKV_ERR_UNSUPPORTED = 2,        /* valid but not implemented (e.g. prefill D=256) */
+  SKV_ERR_WORKSPACE_TOO_SMALL = 3,/* workspace_bytes < the *_workspace() query */
+  SKV_ERR_CUDA = 4                /* a CUDA runtime/driver call failed; see skv_last_cuda_error */
+} skv_status;
+
+typedef enum { SKV_BF16 = 0, SKV_FP16 = 1, SKV_FP32 = 2 } skv_dtype;
+
+/* HND: [B, H, S, D] contiguous.  NHD: [B, S, H, D] contiguous.
+ * TND: packed varlen [T, H, D] contiguous; needs cu_seqlens. */
+typedef enum { SKV_HND = 0, SKV_NHD = 1, SKV_TND = 2 } skv_layout;
+
+/* ------------------------------------------------------------------------ */
+/* attn_fwd_lse: attention forward with a per-row log2 LSE (prefill/varlen). */
+/*
+ * Defined by the ARK return_lse issue ("Expected:" and the repro's
+ * ref_lse_log2); layouts and the varlen LSE shape by the SGLang sgl_kernel::fwd
+ * PR (CUDA FA: varlen LSE 2-D, dense 3-D); GQA by Hq % Hkv == 0 (SGLang Ascend
+ * backend record, validationCode), query head h reading kv head h / (Hq/Hkv).
+ *
+ * Dense (layout HND or NHD; cu_seqlens_q = cu_seqlens_k = NULL):
+ *   q [B, Hq, Sq, D] / [B, Sq, Hq, D]; k, v [B, Hkv, Sk, D] / [B, Sk, Hkv, D];
+ *   out like q; lse [B, Hq, Sq] fp32 (nullable).
+ * Varlen (layout TND): B = number of sequences; cu_seqlens_q, cu_seqlens_k are
+ *   DEVICE int32 arrays of B+1 non-decreasing offsets starting at 0;
+ *   q [total_q, Hq, D], k, v [total_k, Hkv, D] with total_q = Sq and
+ *   total_k = Sk (the caller passes the packed totals); sequence b owns query
+ *   rows [cu_q[b], cu_q[b+1]) and keys [cu_k[b], cu_k[b+1]); out like q;
+ *   lse [Hq, total_q] (nullable).  max_seqlen_q bounds every query length
+ *   (used to size the grid); max_seqlen_k is accepted for API symmetry.
+ * Non-causal: every query row sees every key of its sequence.
+ *
+ * smooth_k != 0: before the product, K is replaced by K' = K - mean(K) with the
+ * mean taken in fp32 over the call's own KV range, per (batch or sequence,
+ * kv head, channel), rounded back to the input type; the LSE is corrected by
+ * adding scale * (q_i . mean(K)) / ln 2, so it stays the LSE of the ORIGINAL
+ * logits (ARK issue, second issue and part 3 of the repro).  O is unchanged up
+ * to rounding (softmax is shift invariant).  Needs workspace (see below).
+ *
+ * scale: the logit scale (e.g. D^-0.5), finite.
+ * workspace: device, >= attn_fwd_lse_workspace(...) bytes, 256-byte aligned;
+ *   may be NULL when that query returns 0.  After a varlen call its first
+ *   bytes hold the work order: int32 order[B] (sequences, longest kv first,
+ *   ties by index) then int32 offsets[B+1] (prefix sums of Hq*ceil(len_q/256)).
+ * Errors: SKV_ERR_INVALID_ARG for NULL q/k/v/out, non-positive sizes (B, Hq,
+ *   Hkv, D; Sq, Sk may be 0 in the dense case), Hq % Hkv != 0, misaligned
+ *   pointers, unknown layout/dtype, or missing/extra cu_seqlens;
+ *   SKV_ERR_UNSUPPORTED for D not in {64,128} or dtype fp32.
+ */
+skv_status attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                        skv_dtype dtype, skv_layout layout,
+                        const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                        int max_seqlen_q, int max_seqlen_k, int smooth_k,
+                        void* workspace, size_t workspace_bytes, skv_stream_t stream);
+
+/* Workspace bytes attn_fwd_lse needs for these arguments (0 if none).
+ * Sk is the per-batch key length (dense) or total_k (TND). Host-only, pure. */
+size_t attn_fwd_lse_workspace(int B, int Hq, int Hkv, int Sk, int D, skv_dtype dtype,
+                              skv_layout layout, int smooth_k);
+
+/* Host restatement of the varlen work order the device builds (for tests and
+ * inspection).  cu_seqlens_q/k are HOST arrays of B+1 entries; writes order[B]
+ * and offsets[B+1] as documented under attn_fwd_lse with rows_per_cta = 256. */
+skv_status attn_varlen_plan(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                            int Hq, int32_t* order, int32_t* offsets);
+
+/* ------------------------------------------------------------------------ */
+/* attn_splitkv_decode: split-KV decode with a stable online softmax.        */
+/*
+ * ExecuTorch PR #22133 (split-K decode kernel, small-query split-K kernel and
+ * cross-split reduce; review items 1-3): each split keeps its own running max
+ * and writes rescaled partials; the partials are merged against the global
+ * max.  Empty trailing splits are allowed and write O = 0, LSE = -inf.
+ *
+ * q [B, Hq, Lq, D]; k, v [B, Hkv, Lkv, D] (HND, contiguous); out [B, Hq, Lq, D];
+ * lse [B, Hq, Lq] fp32 (nullable).  1 <= Lq (any Lq works; 1..4 is the target).
+ * Non-causal: all Lq rows see keys [0, kv_len[b]).
+ * kv_len: DEVICE int32 [B] or NULL (= Lkv for every batch).  It is read on the
+ *   device, so a captured CUDA graph follows its current value; values are
+ *   clamped to [0, Lkv].
+ * num_splits: 0 = automatic (attn_splitkv_plan with the device's SM count);
+ *   otherwise the number of splits, 1..256.
+ * workspace: device, >= attn_splitkv_workspace(B, Hq, Lq, D, num_splits) bytes
+ *   for the split count actually used (0 bytes when it is 1).
+ * Errors as for attn_fwd_lse; SKV_ERR_UNSUPPORTED for D not in {64,128,256}.
+ */
+skv_status attn_splitkv_decode(const void* q, const void* k, const void* v, void* out,
+                               float* lse, int B, int Hq, int Hkv, int Lq, int Lkv, int D,
+                               float scale, skv_dtype dtype, const int32_t* kv_len,
+                               int num_splits, void* workspace, size_t workspace_bytes,
+                               skv_stream_t stream);
+
+/* Split plan (host, pure integer).  For n keys, split s covers
+ *   [s*C, min((s+1)*C, n)),  C = 64 * ceil(ceil(n / num_splits) / 64).
+ * If requested_splits > 0 it is used as is (1..256); otherwise the count is
+ * chosen to give every one of num_sms SMs two CTAs (CTAs = B * Hkv *
+ * ceil(G*Lq/16) * splits, G = Hq/Hkv), keeping >= 128 keys per split, at most
+ * 256 splits, and none that the rounding of C would leave empty.
+ * Writes *num_splits and, if bounds != NULL, bounds[0..num_splits] (host) with
+ * split s = [bounds[s], bounds[s+1]). */
+skv_status attn_splitkv_plan(int B, int Hq, int Hkv, int Lq, int n, int num_sms,
+                             int requested_splits, int* num_splits, int32_t* bounds);
+
+/* Workspace bytes for a decode with this many splits (fp32 partial O and LSE). */
+size_t attn_splitkv_workspace(int B, int Hq, int Lq, int D, int num_splits);
+
+/* ------------------------------------------------------------------------ */
+/* merge_state: combine P partial (O, LSE) results of disjoint KV ranges.    */
+/*
+ * The per-hop merge of ring attention (merge_state_v2 / _merge_attention_partials
+ * in the SGLang PR thread) and the cross-split reduce of the ExecuTorch split-K
+ * PR: per row, M = max_p L_p, w_p = 2^(L_p - M) (0 for -inf),
+ *   O = sum_p w_p O_p / sum_p w_p,  LSE = M + log2(sum_p w_p);
+ * if every part is -inf: O = 0, LSE = -inf.  Parts of weight 0 are not read.
+ *
+ * o_parts: device, P parts each laid out like an attention output of shape
+ *   (B, H, S, D) in `layout` (HND: [B,H,S,D]; NHD/TND: [B,S,H,D], for TND pass
+ *   B = 1 and S = total_q); part p starts part_stride_o ELEMENTS after part p-1
+ *   (0 = B*H*S*D, i.e. packed).
+ * lse_parts: device fp32, P parts of [B, H, S] (for TND: [H, total_q]);
+ *   part stride part_stride_lse elements (0 = B*H*S).
+ * out: device, one part's layout, type out_dtype; lse: device [B,H,S] or NULL.
+ * parts_dtype: bf16, fp16 or fp32; out_dtype: bf16, fp16 or fp32.
+ * Any flattening of rows works with B = H = 1, S = rows, layout HND.
+ */
+skv_status merge_state(const void* o_parts, const float* lse_parts, void* out, float* lse,
+                       int P, int B, int H, int S, int D, skv_layout layout,
+                       skv_dtype parts_dtype, skv_dtype out_dtype,
+                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Diagnostics.                                                              */
+
+/* Static text for a status code. */
+const char* skv_status_string(skv_status s);
+
+/* The cudaError_t of the last failing CUDA call made by this library on the
+ * calling host thread (0 if none). */
+int skv_last_cuda_error(void);
+
+/* Reads and clears the device-side error word of the current device: nonzero if
+ * a kernel gave up a bounded pipeline wait (it then returns without hanging; its
+ * outputs are undefined).  Synchronises the device.  Returns SKV_ERR_CUDA if the
+ * read itself fails. */
+skv_status skv_device_error(int* code);
+
+/* Library version, e.g. "0.1.0". */
+const char* skv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPLITKV_H_ */

@@ -1,0 +1,369 @@
+// Split-KV decode kernel (memory bound): per (batch, kv head, row group,
+// split) one CTA streams its split of K and V from HBM exactly once.
+//
+// Prior art: the ExecuTorch split-K decode kernels (PR #22133, "Prevent
+// Voxtral NaNs in CUDA split-K attention").  That PR replaced a fixed
+// exponent offset by a per-split running max with rescaled partials; this
+// kernel does the same (stable online softmax in the exp2 domain), writes
+// every partial slot (empty splits write O = 0, LSE = -inf) and leaves the
+// cross-split reduction to the merge_state kernel.
+//
+// B200 mapping:
+//  * the G*Lq query rows that share one kv head (GQA) form one 16-row M tile,
+//    so each K/V byte read from HBM serves all of them;
+//  * one producer warp streams 64-key K and V tiles with 2-D TMA loads
+//    (128-byte swizzle, no multicast) into an NS-stage mbarrier ring;
+//  * four consumer warps each take 16 keys of every tile and run
+//    S = Q K^T and O += P V as m16n8k16 tensor-core MMAs (fp32 accumulate)
+//    with the online softmax in registers; warp states are combined through
+//    shared memory at the end.
+// Tensor cores are used because at G*Lq = 16 rows the FMA work per key
+// (2 * 16 * D) exceeds what the CUDA cores sustain at HBM rate; the MMA shape
+// simply holds the 16 rows that share a kv head.
+#pragma once
+
+#include "skv_device.cuh"
+
+namespace skv {
+
+constexpr int kDecodeKeysPerTile = 64;
+constexpr int kDecodeRows = 16;
+constexpr int kDecodeConsumerWarps = 4;
+constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
+
+template <int D>
+struct DecodeCfg {
+  static constexpr int kBoxes = D / 64;                       // 64-element column boxes per row
+  static constexpr int kTileBytes = kBoxes * kDecodeKeysPerTile * 128;  // one K or V tile
+  static constexpr int kStages = (D == 64) ? 6 : 3;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kQStride = D + 8;                      // elements; 16-byte pad per row
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kCombineBytes = kDecodeConsumerWarps * kDecodeRows * (D + 2) * 4;
+  static_assert(kRingBytes >= kCombineBytes, "combine area reuses the ring");
+  static constexpr int kQBytes = kDecodeRows * kQStride * 2;
+  static constexpr int kSmemBytes = kRingBytes + kQBytes + 2 * kStages * 8 + 16 + 1024;  // +align pad
+  static constexpr bool kQInRegs = (D <= 128);
+};
+
+struct DecodeArgs {
+  const void* q;
+  void* out;
+  float* lse;
+  float* part_o;
+  float* part_lse;
+  const int* kv_len;
+  int B, Hq, Hkv, Lq, Lkv;
+  int num_splits;
+  int row_groups;
+  float scale_log2;
+};
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                      const __grid_constant__ CUtensorMap tmV,
+                                                                      const DecodeArgs a) {
+  using Cfg = DecodeCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  T* qs = reinterpret_cast<T*>(smem + Cfg::kRingBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kRingBytes + Cfg::kQBytes);
+  uint64_t* empty = full + Cfg::kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + Cfg::kStages);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int split = blockIdx.x;
+  const int G = a.Hq / a.Hkv;
+  const int rows_total = G * a.Lq;
+  const int rg = blockIdx.y % a.row_groups;
+  const int hkv = (blockIdx.y / a.row_groups) % a.Hkv;
+  const int b = blockIdx.y / (a.row_groups * a.Hkv);
+
+  // ---- split bounds (same rule as the host planner)
+  int n = a.Lkv;
+  if (a.kv_len != nullptr) n = min(max(a.kv_len[b], 0), a.Lkv);
+  int s0 = 0, s1 = 0;
+  if (n > 0) {
+    const int per = (n + a.num_splits - 1) / a.num_splits;
+    const int C = ((per + 63) / 64) * 64;
+    s0 = min(split * C, n);
+    s1 = min(s0 + C, n);
+  }
+  const int ntiles = (s1 - s0 + kDecodeKeysPerTile - 1) / kDecodeKeysPerTile;
+
+  if (tid == 0) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDecodeConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // ---- Q rows of this group into shared memory (zero rows pad the tile)
+  {
+    constexpr int vpr = D / 8;
+    for (int v = tid; v < kDecodeRows * vpr; v += kDecodeThreads) {
+      const int r = v / vpr, c = v % vpr;
+      const int rglob = rg * kDecodeRows + r;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (rglob < rows_total) {
+        const int h = hkv * G + rglob / a.Lq;
+        const int i = rglob % a.Lq;
+        const T* src = static_cast<const T*>(a.q) + ((static_cast<int64_t>(b) * a.Hq + h) * a.Lq + i) * D + c * 8;
+        val = *reinterpret_cast<const uint4*>(src);
+      }
+      *reinterpret_cast<uint4*>(qs + r * Cfg::kQStride + c * 8) = val;
+    }
+  }
+  __syncthreads();
+
+  const int64_t row0 = (static_cast<int64_t>(b) * a.Hkv + hkv) * a.Lkv;
+
+  if (warp == kDecodeConsumerWarps) {
+    // ================= producer warp: TMA ring
+    if (lane == 0 && ntiles > 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      int issued = 0;
+      for (int t = 0; t < ntiles; ++t) {
+        const int st = t % Cfg::kStages;
+        if (t >= Cfg::kStages) {
+          if (!mbar_wait(&empty[st], ((t / Cfg::kStages) & 1) ^ 1, abort_flag, 0x101)) break;
+        }
+        mbar_arrive_expect_tx(&full[st], Cfg::kStageBytes);
+        uint8_t* kt = ring + st * Cfg::kStageBytes;
+        uint8_t* vt = kt + Cfg::kTileBytes;
+        const int row = static_cast<int>(row0 + s0 + t * kDecodeKeysPerTile);
+#pragma unroll
+        for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+          tma_load_2d(kt + bx * kDecodeKeysPerTile * 128, &tmK, &full[st], bx * 64, row);
+          tma_load_2d(vt + bx * kDecodeKeysPerTile * 128, &tmV, &full[st], bx * 64, row);
+        }
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        // let every load already issued land before the CTA's shared memory goes away
+        for (int t = max(0, issued - Cfg::kStages); t < issued; ++t)
+          mbar_drain(&full[t % Cfg::kStages], (t / Cfg::kStages) & 1, 20000000ull);
+      }
+    }
+    return;
+  }
+
+  // ================= consumer warps
+  const int g = lane >> 2, tq = lane & 3;
+  const uint32_t qs_addr = smem_u32(qs);
+  uint32_t qa[Cfg::kQInRegs ? D / 16 : 1][4];
+  if constexpr (Cfg::kQInRegs) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int c = kk * 16 + (lane >> 4) * 8;
+      ldmatrix_x4(qs_addr + (r * Cfg::kQStride + c) * 2, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+    }
+  }
+  float m[2] = {-INFINITY, -INFINITY};
+  float lsum[2] = {0.f, 0.f};
+  float o[D / 8][4];
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+
+  bool ok = true;
+  for (int t = 0; t < ntiles; ++t) {
+    const int st = t % Cfg::kStages;
+    if (!mbar_wait(&full[st], (t / Cfg::kStages) & 1, abort_flag, 0x102)) { ok = false; break; }
+    const uint32_t kt = smem_u32(ring + st * Cfg::kStageBytes);
+    const uint32_t vt = kt + Cfg::kTileBytes;
+    const int key0 = s0 + t * kDecodeKeysPerTile + warp * 16;  // first key of this warp
+    const int nvalid = min(16, s1 - key0);                     // may be <= 0
+
+    // ---- S = Q K^T for 16 rows x 16 keys
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t aq[4];
+      if constexpr (Cfg::kQInRegs) {
+        aq[0] = qa[kk][0]; aq[1] = qa[kk][1]; aq[2] = qa[kk][2]; aq[3] = qa[kk][3];
+      } else {
+        const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int c = kk * 16 + (lane >> 4) * 8;
+        ldmatrix_x4(qs_addr + (r * Cfg::kQStride + c) * 2, aq[0], aq[1], aq[2], aq[3]);
+      }
+      const int bx = kk >> 2;
+      const int chunk = (kk & 3) * 2 + ((lane >> 3) & 1);
+      const int krow = warp * 16 + (lane & 7) + (lane >> 4) * 8;
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4(kt + bx * kDecodeKeysPerTile * 128 + sw128(krow, chunk), b0, b1, b2, b3);
+      mma_16816<T>(sc[0], aq, b0, b1);
+      mma_16816<T>(sc[1], aq, b2, b3);
+    }
+
+    // ---- online softmax (exp2 domain), rows g and g+8 of the tile
+    float x[2][4];
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kidx = nt * 8 + 2 * tq + (e & 1);
+        const float val = (kidx < nvalid) ? sc[nt][e] * a.scale_log2 : -INFINITY;
+        x[nt][e] = val;
+      }
+      mx0 = fmaxf(mx0, fmaxf(x[nt][0], x[nt][1]));
+      mx1 = fmaxf(mx1, fmaxf(x[nt][2], x[nt][3]));
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+    const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
+    const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
+    const float al0 = ex2_approx(m[0] - mu0), al1 = ex2_approx(m[1] - mu1);
+    m[0] = mn0;
+    m[1] = mn1;
+    float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      x[nt][0] = ex2_approx(x[nt][0] - mu0);
+      x[nt][1] = ex2_approx(x[nt][1] - mu0);
+      x[nt][2] = ex2_approx(x[nt][2] - mu1);
+      x[nt][3] = ex2_approx(x[nt][3] - mu1);
+      ps0 += x[nt][0] + x[nt][1];
+      ps1 += x[nt][2] + x[nt][3];
+    }
+    lsum[0] = lsum[0] * al0 + ps0;
+    lsum[1] = lsum[1] * al1 + ps1;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+      o[j][0] *= al0; o[j][1] *= al0;
+      o[j][2] *= al1; o[j][3] *= al1;
+    }
+    uint32_t pa[4];
+    pa[0] = pack2<T>(x[0][0], x[0][1]);
+    pa[1] = pack2<T>(x[0][2], x[0][3]);
+    pa[2] = pack2<T>(x[1][0], x[1][1]);
+    pa[3] = pack2<T>(x[1][2], x[1][3]);
+
+    // keys past the end of the split: their P is 0, and their V rows (which
+    // may hold anything, e.g. unfilled cache) are zeroed so 0 * V stays 0
+    if (nvalid < 16) {
+      const int nz = 16 - max(nvalid, 0);
+      uint8_t* vgen = ring + st * Cfg::kStageBytes + Cfg::kTileBytes;
+      for (int idx = lane; idx < nz * Cfg::kBoxes * 8; idx += 32) {
+        const int rr = 16 - nz + idx / (Cfg::kBoxes * 8);
+        const int rem = idx % (Cfg::kBoxes * 8);
+        const int bx = rem / 8, ch = rem % 8;
+        *reinterpret_cast<uint4*>(vgen + bx * kDecodeKeysPerTile * 128 + (warp * 16 + rr) * 128 + ch * 16) =
+            make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+    }
+
+    // ---- O += P V
+#pragma unroll
+    for (int nd = 0; nd < D / 16; ++nd) {
+      const int bx = nd >> 2;
+      const int chunk = (nd & 3) * 2 + (lane >> 4);
+      const int vrow = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      uint32_t v0, v1, v2, v3;
+      ldmatrix_x4_trans(vt + bx * kDecodeKeysPerTile * 128 + sw128(vrow, chunk), v0, v1, v2, v3);
+      mma_16816<T>(o[2 * nd], pa, v0, v1);
+      mma_16816<T>(o[2 * nd + 1], pa, v2, v3);
+    }
+    if (nvalid < 16) fence_proxy_async_smem();  // generic writes before the async proxy reuses the stage
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+
+  // ---- combine the four warps' states
+  named_barrier_sync(1, kDecodeConsumerWarps * 32);
+  if (!ok || *abort_flag) return;
+  lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], 1);
+  lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], 2);
+  lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], 1);
+  lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], 2);
+  float* cm = reinterpret_cast<float*>(ring);                    // [4][16] running max
+  float* cl = cm + kDecodeConsumerWarps * kDecodeRows;            // [4][16] sums
+  float* co = cl + kDecodeConsumerWarps * kDecodeRows;            // [4][16][D] accumulators
+  if (tq == 0) {
+    cm[warp * 16 + g] = m[0];
+    cm[warp * 16 + g + 8] = m[1];
+    cl[warp * 16 + g] = lsum[0];
+    cl[warp * 16 + g + 8] = lsum[1];
+  }
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j) {
+    const int d = j * 8 + 2 * tq;
+    *reinterpret_cast<float2*>(co + (warp * 16 + g) * D + d) = make_float2(o[j][0], o[j][1]);
+    *reinterpret_cast<float2*>(co + (warp * 16 + g + 8) * D + d) = make_float2(o[j][2], o[j][3]);
+  }
+  named_barrier_sync(1, kDecodeConsumerWarps * 32);
+
+  // 128 threads: 8 per row, each a D/8 slice
+  const int r = tid >> 3;
+  const int sl = tid & 7;
+  const int rglob = rg * kDecodeRows + r;
+  if (rglob >= rows_total) return;
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kDecodeConsumerWarps; ++w) M = fmaxf(M, cm[w * 16 + r]);
+  float e[kDecodeConsumerWarps];
+  float L = 0.f;
+#pragma unroll
+  for (int w = 0; w < kDecodeConsumerWarps; ++w) {
+    const float mw = cm[w * 16 + r];
+    e[w] = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
+    L += e[w] * cl[w * 16 + r];
+  }
+  const float inv = (L > 0.f) ? 1.0f / L : 0.f;
+  const float lse_val = (L > 0.f) ? M + __log2f(L) : -INFINITY;
+  const int h = hkv * G + rglob / a.Lq;
+  const int i = rglob % a.Lq;
+  const int64_t orow = (static_cast<int64_t>(b) * a.Hq + h) * a.Lq + i;
+  const int64_t rows_all = static_cast<int64_t>(a.B) * a.Hq * a.Lq;
+  constexpr int per = D / 8;
+  if (a.num_splits == 1) {
+    T* dst = static_cast<T*>(a.out) + orow * D + sl * per;
+#pragma unroll
+    for (int c = 0; c < per; c += 8) {
+      float v[8];
+#pragma unroll
+      for (int q2 = 0; q2 < 8; ++q2) {
+        const int d = sl * per + c + q2;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecodeConsumerWarps; ++w) acc = fmaf(e[w], co[(w * 16 + r) * D + d], acc);
+        v[q2] = acc * inv;
+      }
+      uint4 u;
+      u.x = pack2<T>(v[0], v[1]);
+      u.y = pack2<T>(v[2], v[3]);
+      u.z = pack2<T>(v[4], v[5]);
+      u.w = pack2<T>(v[6], v[7]);
+      *reinterpret_cast<uint4*>(dst + c) = u;
+    }
+    if (sl == 0 && a.lse != nullptr) a.lse[orow] = lse_val;
+  } else {
+    float* dst = a.part_o + (static_cast<int64_t>(split) * rows_all + orow) * D + sl * per;
+#pragma unroll
+    for (int c = 0; c < per; c += 4) {
+      float v[4];
+#pragma unroll
+      for (int q2 = 0; q2 < 4; ++q2) {
+        const int d = sl * per + c + q2;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecodeConsumerWarps; ++w) acc = fmaf(e[w], co[(w * 16 + r) * D + d], acc);
+        v[q2] = acc * inv;
+      }
+      *reinterpret_cast<float4*>(dst + c) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+    if (sl == 0) a.part_lse[static_cast<int64_t>(split) * rows_all + orow] = lse_val;
+  }
+}
+
+}  // namespace skv

@@ -1,0 +1,486 @@
+// Prefill / varlen attention forward with a per-row log2 LSE on sm_100a.
+//
+// Defines O_i = softmax_j(scale * q_i . k_j) V and LSE_i = log2 sum_j exp(scale *
+// q_i . k_j) over the original logits, one LSE per row (ARK return_lse issue,
+// "Expected:").  The ARK kernel the issue describes stored one value per
+// 16-row group; here the softmax thread that owns TMEM lane i (= query row i
+// of its 128-row tile) computes and stores row i's LSE itself.
+//
+// CTA = up to two 128-row query tiles of one (sequence, head) that share every
+// K/V tile.  Warp roles (320 threads):
+//   warps 0-3  softmax + epilogue for query tile 0 (thread t owns row t)
+//   warps 4-7  softmax + epilogue for query tile 1
+//   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of
+//              NS shared-memory buffers (128-byte swizzle, no multicast)
+//   warp  9    TMEM allocator and (one elected thread) tcgen05.mma issuer
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
+// O_1 [256+D, 256+2D).  S_a holds fp32 logits; the softmax writes P_a as
+// packed 16-bit pairs into S_a's first 64 columns, and O_a += P_a V_j reads P_a
+// straight from TMEM (A operand in tensor memory).
+//
+// Per KV tile j the MMA thread issues PV_0(j), PV_1(j), then S_0(j+1),
+// S_1(j+1).  The next S into S_a overwrites P_a, which PV_a(j) reads; the PTX
+// ISA orders consecutive MMAs only when they share an accumulator, so the MMA
+// thread waits for PV_a(j) to complete (its own commit barrier) before issuing
+// S_a(j+1); the other tile's MMA keeps the tensor pipe busy meanwhile.
+//
+// Online softmax in the exp2 domain with a lazily updated running max: the
+// max is only raised (and O_a rescaled in TMEM) when it grows by more than 8
+// (log2 units); otherwise the stale max is kept, which bounds P by 2^8 and is
+// exact once O and the row sum are divided at the end.  No fixed exponent
+// offset is used anywhere (ExecuTorch split-K PR).
+#pragma once
+
+#include <type_traits>
+
+#include "skv_device.cuh"
+#include "tcgen05.cuh"
+
+namespace skv {
+
+constexpr int kPfBM = 128;          // rows per query tile
+constexpr int kPfBN = 128;          // keys per KV tile
+constexpr int kPfThreads = 320;
+constexpr float kPfRescaleThreshold = 8.0f;
+
+template <int D>
+struct PrefillCfg {
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kBoxBytes = 128 * 128;       // 128 rows x 128 bytes
+  static constexpr int kQTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kKVTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kStages = (D == 64) ? 8 : 4;
+  static constexpr int kRingBytes = kStages * kKVTileBytes;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffRing = 2 * kQTileBytes;
+  static constexpr int kOffBar = kOffRing + kRingBytes;
+  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], o_full[2], drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 * 4 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + TMEM slot, abort flag; + alignment pad
+  static constexpr int kSCol0 = 0, kSCol1 = 128, kOCol0 = 256, kOCol1 = 256 + D;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+struct PrefillArgs {
+  void* out;
+  float* lse;
+  const float* kmean;   // smooth: [Bseq, Hkv, D] fp32, else null
+  const int* cu_q;
+  const int* cu_k;
+  const int* order;
+  const int* offsets;
+  int B, Hq, Hkv, Sq, Sk;
+  int nqb;              // dense: 256-row query blocks per (b, h)
+  int layout;           // 0 HND, 1 NHD, 2 TND
+  float scale_log2;
+};
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
+  using Cfg = PrefillCfg<D>;
+  constexpr int kIsBf16 = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
+  constexpr uint32_t kIdescQK = tc5::idesc_f16(kIsBf16, 0, kPfBM, kPfBN);
+  constexpr uint32_t kIdescPV = tc5::idesc_f16(kIsBf16, 1, kPfBM, D);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + Cfg::kStages;
+  uint64_t* s_full = kv_empty + Cfg::kStages;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* o_full = pv_done + 2;
+  uint64_t* drain = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 8);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int G = a.Hq / a.Hkv;
+
+  // ---------------- work item
+  int b, h, qblk, len_q, len_k, q_row0, k_row0, bcoord;
+  if (a.layout == 2) {
+    const int item = blockIdx.x;
+    if (item >= a.offsets[a.B]) return;
+    int lo = 0, hi = a.B - 1;  // last p with offsets[p] <= item
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.offsets[mid] <= item) lo = mid; else hi = mid - 1;
+    }
+    b = a.order[lo];
+    const int rem = item - a.offsets[lo];
+    len_q = a.cu_q[b + 1] - a.cu_q[b];
+    len_k = a.cu_k[b + 1] - a.cu_k[b];
+    const int nblk = (len_q + 2 * kPfBM - 1) / (2 * kPfBM);
+    h = rem / nblk;
+    qblk = rem % nblk;
+    q_row0 = a.cu_q[b] + qblk * 2 * kPfBM;
+    k_row0 = a.cu_k[b];
+    bcoord = 0;
+  } else {
+    const int item = blockIdx.x;
+    qblk = item % a.nqb;
+    h = (item / a.nqb) % a.Hq;
+    b = item / (a.nqb * a.Hq);
+    len_q = a.Sq;
+    len_k = a.Sk;
+    q_row0 = qblk * 2 * kPfBM;
+    k_row0 = 0;
+    bcoord = b;
+  }
+  const int hkv = h / G;
+  const int rows_here = min(2 * kPfBM, len_q - qblk * 2 * kPfBM);
+  const int nt = rows_here > kPfBM ? 2 : 1;
+  const int nkv = (len_k + kPfBN - 1) / kPfBN;
+
+  // output addressing for query row qi (index inside the sequence)
+  auto out_row = [&](int qi) -> T* {
+    int64_t r;
+    if (a.layout == 0) r = (static_cast<int64_t>(b) * a.Hq + h) * a.Sq + qi;
+    else if (a.layout == 1) r = (static_cast<int64_t>(b) * a.Sq + qi) * a.Hq + h;
+    else r = static_cast<int64_t>(a.cu_q[b] + qi) * a.Hq + h;
+    return static_cast<T*>(a.out) + r * D;
+  };
+  auto lse_idx = [&](int qi) -> int64_t {
+    if (a.layout == 2) return static_cast<int64_t>(h) * a.Sq + a.cu_q[b] + qi;
+    return (static_cast<int64_t>(b) * a.Hq + h) * a.Sq + qi;
+  };
+
+  if (nkv == 0) {
+    // no keys: O = 0, LSE = -inf for every valid row of this block
+    for (int r = tid; r < rows_here; r += kPfThreads) {
+      const int qi = qblk * 2 * kPfBM + r;
+      uint4* dst = reinterpret_cast<uint4*>(out_row(qi));
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+      if (a.lse != nullptr) a.lse[lse_idx(qi)] = -INFINITY;
+    }
+    return;
+  }
+
+  // ---------------- setup
+  if (tid == 0) {
+    for (int i = 0; i < Cfg::kNumBars; ++i) mbar_init(&bars[i], (&bars[i] == &p_full[0] || &bars[i] == &p_full[1]) ? 128u : 1u);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tc5::alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tc5::relinquish();
+  }
+  tc5::fence_before();
+  __syncthreads();
+  tc5::fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  uint8_t* qtile[2] = {smem + Cfg::kOffQ, smem + Cfg::kOffQ + Cfg::kQTileBytes};
+  uint8_t* ring = smem + Cfg::kOffRing;
+
+  if (warp == 8) {
+    // ======================= TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const bool hnd = (a.layout == 0);
+      mbar_arrive_expect_tx(q_full, nt * Cfg::kQTileBytes);
+      for (int t = 0; t < nt; ++t) {
+        const int s = q_row0 + t * kPfBM;
+#pragma unroll
+        for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+          if (hnd) tma_load_4d(qtile[t] + bx * Cfg::kBoxBytes, &tmQ, q_full, bx * 64, s, h, bcoord);
+          else tma_load_4d(qtile[t] + bx * Cfg::kBoxBytes, &tmQ, q_full, bx * 64, h, s, bcoord);
+        }
+      }
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = k_row0 + j * kPfBN;
+        for (int which = 0; which < 2; ++which) {
+          const int u = 2 * j + which;
+          const int buf = u % Cfg::kStages;
+          if (u >= Cfg::kStages) {
+            if (!mbar_wait(&kv_empty[buf], ((u / Cfg::kStages) & 1) ^ 1, abort_flag, kErrPrefillWait)) {
+              ok = false;
+              break;
+            }
+          }
+          mbar_arrive_expect_tx(&kv_full[buf], Cfg::kKVTileBytes);
+          const CUtensorMap* m = which ? &tmV : &tmK;
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+            uint8_t* dst = ring + buf * Cfg::kKVTileBytes + bx * Cfg::kBoxBytes;
+            if (hnd) tma_load_4d(dst, m, &kv_full[buf], bx * 64, s, hkv, bcoord);
+            else tma_load_4d(dst, m, &kv_full[buf], bx * 64, hkv, s, bcoord);
+          }
+          issued = u + 1;
+        }
+      }
+      if (*abort_flag) {
+        mbar_drain(q_full, 0, 20000000ull);
+        for (int u = max(0, issued - Cfg::kStages); u < issued; ++u)
+          mbar_drain(&kv_full[u % Cfg::kStages], (u / Cfg::kStages) & 1, 20000000ull);
+      }
+    }
+  } else if (warp == 9) {
+    // ======================= MMA issuer
+    if (lane == 0) {
+      const uint32_t q_addr[2] = {smem_u32(qtile[0]), smem_u32(qtile[1])};
+      const uint32_t ring_addr = smem_u32(ring);
+      const uint32_t s_col[2] = {tmem + Cfg::kSCol0, tmem + Cfg::kSCol1};
+      const uint32_t o_col[2] = {tmem + Cfg::kOCol0, tmem + Cfg::kOCol1};
+      bool ok = mbar_wait(q_full, 0, abort_flag, kErrPrefillWait);
+      auto issue_s = [&](int t, uint32_t kaddr) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Cfg::kBoxBytes + (kk & 3) * 32;
+          tc5::mma_ss(s_col[t], tc5::smem_desc(q_addr[t] + off, 16, 1024), tc5::smem_desc(kaddr + off, 16, 1024),
+                      kIdescQK, kk > 0 ? 1u : 0u);
+        }
+      };
+      if (ok) {
+        const int buf0 = 0;
+        ok = mbar_wait(&kv_full[buf0], 0, abort_flag, kErrPrefillWait);
+        if (ok) {
+          tc5::fence_after();
+          for (int t = 0; t < nt; ++t) {
+            issue_s(t, ring_addr + buf0 * Cfg::kKVTileBytes);
+            tc5::commit(smem_u32(&s_full[t]));
+          }
+          tc5::commit(smem_u32(&kv_empty[buf0]));
+        }
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int uv = 2 * j + 1;
+        const int bufv = uv % Cfg::kStages;
+        if (!mbar_wait(&kv_full[bufv], (uv / Cfg::kStages) & 1, abort_flag, kErrPrefillWait)) { ok = false; break; }
+        const uint32_t vaddr = ring_addr + bufv * Cfg::kKVTileBytes;
+        for (int t = 0; t < nt; ++t) {
+          if (!mbar_wait(&p_full[t], j & 1, abort_flag, kErrPrefillWait)) { ok = false; break; }
+          tc5::fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kPfBN / 16; ++kk) {
+            tc5::mma_ts(o_col[t], s_col[t] + kk * 8, tc5::smem_desc(vaddr + kk * 2048, Cfg::kBoxBytes, 1024),
+                        kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc5::commit(smem_u32(&pv_done[t]));
+        }
+        if (!ok) break;
+        tc5::commit(smem_u32(&kv_empty[bufv]));
+        if (j + 1 < nkv) {
+          const int uk = 2 * (j + 1);
+          const int bufk = uk % Cfg::kStages;
+          if (!mbar_wait(&kv_full[bufk], (uk / Cfg::kStages) & 1, abort_flag, kErrPrefillWait)) { ok = false; break; }
+          tc5::fence_after();
+          for (int t = 0; t < nt; ++t) {
+            // P_t(j) lives in S_t's columns: PV_t(j) must finish reading it first
+            if (!mbar_wait(&pv_done[t], j & 1, abort_flag, kErrPrefillWait)) { ok = false; break; }
+            tc5::fence_after();
+            issue_s(t, ring_addr + bufk * Cfg::kKVTileBytes);
+            tc5::commit(smem_u32(&s_full[t]));
+          }
+          if (!ok) break;
+          tc5::commit(smem_u32(&kv_empty[bufk]));
+        } else {
+          for (int t = 0; t < nt; ++t) tc5::commit(smem_u32(&o_full[t]));
+        }
+      }
+      // every MMA this thread issued has completed before TMEM is released
+      tc5::commit(smem_u32(drain));
+      mbar_drain(drain, 0, 20000000ull);
+    }
+  } else {
+    // ======================= softmax + epilogue (warps 0-7)
+    const int t = warp >> 2;           // query tile
+    const int lg = warp & 3;           // TMEM lane group
+    const int row = lg * 32 + lane;    // row inside the tile
+    if (t < nt) {
+      const uint32_t lane_base = static_cast<uint32_t>(lg * 32) << 16;
+      const uint32_t s_addr = tmem + lane_base + (t == 0 ? Cfg::kSCol0 : Cfg::kSCol1);
+      const uint32_t o_addr = tmem + lane_base + (t == 0 ? Cfg::kOCol0 : Cfg::kOCol1);
+      const int qi = qblk * 2 * kPfBM + t * kPfBM + row;  // row index inside the sequence
+      const bool row_valid = qi < len_q;
+      bool ok = true;
+
+      // smooth_k: delta = scale*log2(e) * (q_i . mean(K)), the shift smoothing removes
+      float delta = 0.f;
+      if (a.kmean != nullptr) {
+        ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, kErrPrefillWait));
+        if (ok) {
+          const float* mu = a.kmean + (static_cast<int64_t>(b) * a.Hkv + hkv) * D;
+          float acc = 0.f;
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+            const uint8_t* qrow = qtile[t] + bx * Cfg::kBoxBytes;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint4 u = *reinterpret_cast<const uint4*>(qrow + sw128(row, c));
+              const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = unpack2<T>(w[e]);
+                const int d = bx * 64 + c * 8 + 2 * e;
+                acc = fmaf(f.x, __ldg(mu + d), acc);
+                acc = fmaf(f.y, __ldg(mu + d + 1), acc);
+              }
+            }
+          }
+          delta = acc * a.scale_log2;
+        }
+      }
+
+      float m_run = -INFINITY;  // running max of the (smoothed) log2-domain logits, possibly stale
+      float l_run = 0.f;
+      for (int j = 0; j < nkv && ok; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, kErrPrefillWait));
+        if (!ok) break;
+        tc5::fence_after();
+        float s[kPfBN];
+#pragma unroll
+        for (int c = 0; c < kPfBN / 32; ++c) {
+          float (&chunk)[32] = *reinterpret_cast<float(*)[32]>(&s[c * 32]);
+          tc5::ld32(s_addr + c * 32, chunk);
+        }
+        tc5::wait_ld();
+        const int n_valid = len_k - j * kPfBN;
+        if (n_valid < kPfBN) {
+#pragma unroll
+          for (int c = 0; c < kPfBN; ++c)
+            if (c >= n_valid) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < kPfBN; ++c) mx = fmaxf(mx, s[c]);
+        const float t_max = fmaf(mx, a.scale_log2, -delta);
+        const float m_new = fmaxf(m_run, t_max);
+        const bool rescale = m_new > m_run + kPfRescaleThreshold;
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = ex2_approx(m_run - m_new);
+          m_run = m_new;
+        }
+        l_run *= alpha;
+        const float neg_bias = -(m_run + delta);
+        float psum = 0.f;
+#pragma unroll
+        for (int c = 0; c < kPfBN / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * e], a.scale_log2, neg_bias));
+            const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * e + 1], a.scale_log2, neg_bias));
+            psum += p0 + p1;
+            pk[e] = pack2<T>(p0, p1);
+          }
+          tc5::st16(s_addr + c * 16, pk);
+        }
+        l_run += psum;
+        tc5::wait_st();
+        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+          // O_t holds the PV products of tiles < j (complete: S_t(j) was issued after them)
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tc5::ld32(o_addr + c * 32, o);
+            tc5::wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tc5::st32(o_addr + c * 32, o);
+          }
+          tc5::wait_st();
+        }
+        tc5::fence_before();
+        mbar_arrive(&p_full[t]);
+      }
+
+      // ---------------- epilogue: O / l and LSE for this thread's row
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[t], 0, abort_flag, kErrPrefillWait));
+      if (ok) {
+        tc5::fence_after();
+        const float inv_l = 1.0f / l_run;
+        T* dst = row_valid ? out_row(qi) : nullptr;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tc5::ld32(o_addr + c * 32, o);
+          tc5::wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack2<T>(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
+          if (row_valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            d4[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+            d4[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+          }
+        }
+        if (row_valid && a.lse != nullptr) a.lse[lse_idx(qi)] = m_run + __log2f(l_run) + delta;
+      }
+    }
+  }
+
+  tc5::fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc5::fence_after();
+    tc5::dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+// Device-side varlen planner (one block): orders sequences by kv length,
+// longest first (ties by index), and writes prefix sums of their work items
+// (Hq * ceil(len_q / 256)).  order[B], offsets[B+1].
+__global__ void __launch_bounds__(1024) varlen_plan_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k,
+                                                            int B, int Hq, int* __restrict__ order,
+                                                            int* __restrict__ offsets) {
+  for (int bb = threadIdx.x; bb < B; bb += blockDim.x) {
+    const int lk = cu_k[bb + 1] - cu_k[bb];
+    int rank = 0;
+    for (int o = 0; o < B; ++o) {
+      const int lo = cu_k[o + 1] - cu_k[o];
+      rank += (lo > lk) || (lo == lk && o < bb);
+    }
+    order[rank] = bb;
+  }
+  __syncthreads();
+  // block-wide exclusive scan of item counts in `order`
+  __shared__ int part[1024];
+  const int per = (B + blockDim.x - 1) / blockDim.x;
+  const int beg = min(B, static_cast<int>(threadIdx.x) * per);
+  const int end = min(B, beg + per);
+  int local = 0;
+  for (int i = beg; i < end; ++i) {
+    const int bb = order[i];
+    const int lq = cu_q[bb + 1] - cu_q[bb];
+    local += Hq * ((lq + 2 * kPfBM - 1) / (2 * kPfBM));
+  }
+  part[threadIdx.x] = local;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int i = 0; i < static_cast<int>(blockDim.x); ++i) {
+      const int v = part[i];
+      part[i] = run;
+      run += v;
+    }
+    offsets[B] = run;
+  }
+  __syncthreads();
+  int run = part[threadIdx.x];
+  for (int i = beg; i < end; ++i) {
+    offsets[i] = run;
+    const int bb = order[i];
+    const int lq = cu_q[bb + 1] - cu_q[bb];
+    run += Hq * ((lq + 2 * kPfBM - 1) / (2 * kPfBM));
+  }
+}
+
+}  // namespace skv

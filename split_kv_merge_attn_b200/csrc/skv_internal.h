@@ -1,0 +1,73 @@
+// Internal interface between the host-side ABI layer (validation, planning,
+// workspace layout) and the translation unit that holds the kernels and their
+// launchers.  Not part of the public C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "splitkv.h"
+
+
+namespace skv {
+
+// Device error codes recorded when a bounded wait gives up.
+enum DeviceError : int {
+  kErrDecodeEmptyWait = 0x101,
+  kErrDecodeFullWait = 0x102,
+  kErrPrefillWait = 0x201,
+};
+
+// Constants of the split planner (mirrored by the decode kernel).
+constexpr int kSplitAlign = 64;
+constexpr int kSplitMinKeys = 128;
+constexpr int kSplitMax = 256;
+constexpr int kCtasPerSm = 2;
+constexpr int kDecodeRowsPerCta = 16;
+constexpr int kPrefillRowsPerCta = 256;
+
+inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Launchers (kernels TU).  Return a cudaError_t value (0 = success).
+int sm_count();  // SM count of the current device (cached per device)
+
+int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, float* lse, int P, int B,
+                       int H, int S, int D, int layout_bsh, skv_dtype parts_dt, skv_dtype out_dt,
+                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream);
+
+int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, float* part_o,
+                  float* part_lse, const int32_t* kv_len, int B, int Hq, int Hkv, int Lq, int Lkv, int D,
+                  float scale, skv_dtype dt, int num_splits, skv_stream_t stream);
+
+struct PrefillLaunch {
+  const void* q;
+  const void* k;  // K, or the smoothed K' when smooth_k
+  const void* v;
+  void* out;
+  float* lse;
+  const float* kmean;      // [B(or seqs), Hkv, D] fp32 when smooth_k, else null
+  const int32_t* cu_q;     // device, varlen only
+  const int32_t* cu_k;
+  const int32_t* order;    // device work order (varlen)
+  const int32_t* offsets;
+  int B, Hq, Hkv, Sq, Sk, D;
+  int max_seqlen_q;
+  float scale;
+  skv_dtype dt;
+  skv_layout layout;
+};
+int launch_prefill(const PrefillLaunch& p, skv_stream_t stream);
+
+int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int32_t* order,
+                       int32_t* offsets, skv_stream_t stream);
+
+// smooth_k prepass: fp32 mean over each (batch or sequence, kv head) KV range
+// into kmean [B, Hkv, D] (via per-256-key partial sums in `partial`), and, if
+// k_smoothed != null, K' = K - mean rounded to the input type.
+int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partial, const int32_t* cu_k, int B,
+                    int Hkv, int Sk, int max_len, int D, skv_dtype dt, skv_layout layout, skv_stream_t stream);
+
+int read_and_clear_device_error(int* code);
+
+}  // namespace skv

@@ -1,0 +1,318 @@
+// Kernel translation unit: every device kernel of the library and the host
+// launchers that build their TMA descriptors and grids.  One translation unit
+// so the device error word is a single object per device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "skv_internal.h"
+#include "skv_device.cuh"
+#include "merge_state.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+#include "smooth.cuh"
+
+namespace skv {
+
+int read_and_clear_device_error(int* code) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_skv_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_skv_device_error, &zero, sizeof(int));
+  if (e != cudaSuccess) return e;
+  *code = v;
+  return 0;
+}
+
+// ------------------------------------------------------------ device info
+
+namespace {
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices] = {0};
+std::mutex g_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorNotSupported;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  *out = g_encode;
+  return 0;
+}
+
+CUtensorMapDataType tmap_type(skv_dtype dt) {
+  return dt == SKV_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+}
+
+// Tiled map over a 16-bit tensor of `rank` dims (dims[0] innermost, strides in
+// bytes for dims 1..rank-1), box {64, box1, ...}, 128-byte swizzle, zero fill.
+int make_tmap(CUtensorMap* m, skv_dtype dt, int rank, const void* base, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  int e = get_encoder(&enc);
+  if (e) return e;
+  cuuint64_t gdim[5];
+  cuuint64_t gstr[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) gstr[i] = strides_bytes[i];
+  CUresult r = enc(m, tmap_type(dt), static_cast<cuuint32_t>(rank), const_cast<void*>(base), gdim, gstr, bx, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : static_cast<int>(cudaErrorInvalidValue);
+}
+}  // namespace
+
+int sm_count() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0) return 0;
+  if (dev < kMaxDevices && g_sms[dev] > 0) return g_sms[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < kMaxDevices) g_sms[dev] = n;
+  return n;
+}
+
+// ------------------------------------------------------------ merge_state
+
+int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, float* lse, int P, int B, int H,
+                       int S, int D, int layout_bsh, skv_dtype parts_dt, skv_dtype out_dt,
+                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream) {
+  MergeArgs a;
+  a.o_parts = o_parts;
+  a.lse_parts = lse_parts;
+  a.out = out;
+  a.lse = lse;
+  a.P = P;
+  a.B = B;
+  a.H = H;
+  a.S = S;
+  a.D = D;
+  a.layout_bsh = layout_bsh;
+  a.part_stride_o = part_stride_o;
+  a.part_stride_lse = part_stride_lse;
+  const int64_t rows = static_cast<int64_t>(B) * H * S;
+  a.n_vec = rows * (D / 8);
+  if (a.n_vec == 0) return 0;
+  const int threads = 256;
+  const int sms = sm_count();
+  int64_t blocks = (a.n_vec + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(sms > 0 ? sms : 148) * 8;  // 8 x 256 threads per SM resident
+  if (blocks > cap) blocks = cap;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define SKV_MERGE(TI, TO) merge_state_kernel<TI, TO><<<static_cast<unsigned>(blocks), threads, 0, st>>>(a)
+  if (parts_dt == SKV_FP32 && out_dt == SKV_BF16) SKV_MERGE(float, __nv_bfloat16);
+  else if (parts_dt == SKV_FP32 && out_dt == SKV_FP16) SKV_MERGE(float, __half);
+  else if (parts_dt == SKV_FP32 && out_dt == SKV_FP32) SKV_MERGE(float, float);
+  else if (parts_dt == SKV_BF16 && out_dt == SKV_BF16) SKV_MERGE(__nv_bfloat16, __nv_bfloat16);
+  else if (parts_dt == SKV_BF16 && out_dt == SKV_FP32) SKV_MERGE(__nv_bfloat16, float);
+  else if (parts_dt == SKV_BF16 && out_dt == SKV_FP16) SKV_MERGE(__nv_bfloat16, __half);
+  else if (parts_dt == SKV_FP16 && out_dt == SKV_FP16) SKV_MERGE(__half, __half);
+  else if (parts_dt == SKV_FP16 && out_dt == SKV_FP32) SKV_MERGE(__half, float);
+  else if (parts_dt == SKV_FP16 && out_dt == SKV_BF16) SKV_MERGE(__half, __nv_bfloat16);
+  else return cudaErrorInvalidValue;
+#undef SKV_MERGE
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ decode
+
+namespace {
+template <int D, typename T>
+int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, dim3 grid,
+                    cudaStream_t st) {
+  using Cfg = DecodeCfg<D>;
+  auto kern = decode_split_kernel<D, T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kDecodeThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
+  return cudaGetLastError();
+}
+}  // namespace
+
+int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, float* part_o,
+                  float* part_lse, const int32_t* kv_len, int B, int Hq, int Hkv, int Lq, int Lkv, int D,
+                  float scale, skv_dtype dt, int num_splits, skv_stream_t stream) {
+  const int G = Hq / Hkv;
+  DecodeArgs a;
+  a.q = q;
+  a.out = out;
+  a.lse = lse;
+  a.part_o = part_o;
+  a.part_lse = part_lse;
+  a.kv_len = kv_len;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Lq = Lq;
+  a.Lkv = Lkv;
+  a.num_splits = num_splits;
+  a.row_groups = static_cast<int>(ceil_div64(static_cast<int64_t>(G) * Lq, kDecodeRows));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  // K and V as 2-D [B*Hkv*Lkv rows, D] maps; box = 64 columns x 64 keys
+  CUtensorMap tk, tv;
+  std::memset(&tk, 0, sizeof(tk));
+  std::memset(&tv, 0, sizeof(tv));
+  if (Lkv > 0) {  // with no keys the kernel issues no loads and the maps stay unused
+    const uint64_t dims[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(B) * Hkv * Lkv};
+    const uint64_t strides[1] = {static_cast<uint64_t>(D) * 2};
+    const uint32_t box[2] = {64, kDecodeKeysPerTile};
+    int e = make_tmap(&tk, dt, 2, k, dims, strides, box);
+    if (e) return e;
+    e = make_tmap(&tv, dt, 2, v, dims, strides, box);
+    if (e) return e;
+  }
+  dim3 grid(num_splits, B * Hkv * a.row_groups);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dt == SKV_BF16) {
+    if (D == 64) return launch_decode_t<64, __nv_bfloat16>(tk, tv, a, grid, st);
+    if (D == 128) return launch_decode_t<128, __nv_bfloat16>(tk, tv, a, grid, st);
+    if (D == 256) return launch_decode_t<256, __nv_bfloat16>(tk, tv, a, grid, st);
+  } else {
+    if (D == 64) return launch_decode_t<64, __half>(tk, tv, a, grid, st);
+    if (D == 128) return launch_decode_t<128, __half>(tk, tv, a, grid, st);
+    if (D == 256) return launch_decode_t<256, __half>(tk, tv, a, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------ prefill
+
+namespace {
+// 4-D map over q/k/v of one layout: HND dims (D, S, H, B); NHD / TND dims
+// (D, H, S, B); box = 64 columns x 128 rows of one head.
+int make_qkv_map(CUtensorMap* m, const void* base, skv_dtype dt, skv_layout layout, int B, int H, int S, int D) {
+  const uint64_t e = 2;
+  uint64_t dims[4], strides[3];
+  uint32_t box[4];
+  if (layout == SKV_HND) {
+    dims[0] = D; dims[1] = S; dims[2] = H; dims[3] = B;
+    strides[0] = D * e; strides[1] = static_cast<uint64_t>(S) * D * e; strides[2] = static_cast<uint64_t>(H) * S * D * e;
+    box[0] = 64; box[1] = 128; box[2] = 1; box[3] = 1;
+  } else {
+    dims[0] = D; dims[1] = H; dims[2] = S; dims[3] = B;
+    strides[0] = D * e; strides[1] = static_cast<uint64_t>(H) * D * e; strides[2] = static_cast<uint64_t>(S) * H * D * e;
+    box[0] = 64; box[1] = 1; box[2] = 128; box[3] = 1;
+  }
+  return make_tmap(m, dt, 4, base, dims, strides, box);
+}
+
+template <int D, typename T>
+int launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillArgs& a,
+                     unsigned grid, cudaStream_t st) {
+  using Cfg = PrefillCfg<D>;
+  auto kern = prefill_kernel<D, T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kPfThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+}  // namespace
+
+int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
+  const bool varlen = p.layout == SKV_TND;
+  const int Bm = varlen ? 1 : p.B;       // batch extent of the maps
+  CUtensorMap tq, tk, tv;
+  int e = make_qkv_map(&tq, p.q, p.dt, p.layout, Bm, p.Hq, p.Sq > 0 ? p.Sq : 1, p.D);
+  if (e) return e;
+  std::memset(&tk, 0, sizeof(tk));
+  std::memset(&tv, 0, sizeof(tv));
+  if (p.Sk > 0) {  // with no keys every CTA writes O = 0, LSE = -inf without loads
+    e = make_qkv_map(&tk, p.k, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D);
+    if (e) return e;
+    e = make_qkv_map(&tv, p.v, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D);
+    if (e) return e;
+  }
+  PrefillArgs a;
+  a.out = p.out;
+  a.lse = p.lse;
+  a.kmean = p.kmean;
+  a.cu_q = p.cu_q;
+  a.cu_k = p.cu_k;
+  a.order = p.order;
+  a.offsets = p.offsets;
+  a.B = p.B;
+  a.Hq = p.Hq;
+  a.Hkv = p.Hkv;
+  a.Sq = p.Sq;
+  a.Sk = p.Sk;
+  a.layout = varlen ? 2 : (p.layout == SKV_HND ? 0 : 1);
+  a.scale_log2 = p.scale * 1.4426950408889634f;
+  int64_t grid;
+  if (varlen) {
+    // upper bound on sum_b ceil(len_q(b) / 256); surplus CTAs exit at once
+    a.nqb = 0;
+    grid = static_cast<int64_t>(p.Hq) * (ceil_div64(p.Sq, kPrefillRowsPerCta) + p.B);
+  } else {
+    a.nqb = static_cast<int>(ceil_div64(p.Sq, kPrefillRowsPerCta));
+    grid = static_cast<int64_t>(p.B) * p.Hq * a.nqb;
+  }
+  if (grid <= 0) return 0;
+  if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (p.dt == SKV_BF16) {
+    if (p.D == 64) return launch_prefill_t<64, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+    if (p.D == 128) return launch_prefill_t<128, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+  } else {
+    if (p.D == 64) return launch_prefill_t<64, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+    if (p.D == 128) return launch_prefill_t<128, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int32_t* order, int32_t* offsets,
+                       skv_stream_t stream) {
+  varlen_plan_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(cu_q, cu_k, B, Hq, order, offsets);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ smooth_k
+
+int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partial, const int32_t* cu_k, int B,
+                    int Hkv, int Sk, int max_len, int D, skv_dtype dt, skv_layout layout, skv_stream_t stream) {
+  SmoothArgs a;
+  a.k = k;
+  a.k_out = k_smoothed;
+  a.partial = partial;
+  a.kmean = kmean;
+  a.cu_k = cu_k;
+  a.Bseq = B;
+  a.Hkv = Hkv;
+  a.Sk = Sk;
+  a.D = D;
+  a.nchunks = static_cast<int>(ceil_div64(max_len, kSmoothChunk));
+  a.layout = layout == SKV_HND ? 0 : (layout == SKV_NHD ? 1 : 2);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (a.nchunks > 0) {
+    dim3 grid(a.nchunks, B, Hkv);
+    if (dt == SKV_BF16) kmean_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
+    else kmean_partial_kernel<__half><<<grid, 256, 0, st>>>(a);
+  }
+  kmean_finalize_kernel<<<B * Hkv, D, 0, st>>>(a);
+  if (k_smoothed != nullptr && a.nchunks > 0) {
+    dim3 grid(a.nchunks, B, Hkv);
+    if (dt == SKV_BF16) ksmooth_write_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
+    else ksmooth_write_kernel<__half><<<grid, 256, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace skv
