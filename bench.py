@@ -1,0 +1,554 @@
+#!/usr/bin/env python
+"""Benchmark of the attention-with-LSE hot path on B200.
+
+One step = one pass over every operation of the path at the workloads' full
+sizes, inputs resident in HBM:
+  * varlen TND prefill, H=24, D=128, seqlens {512,1024,2048,4096}   (attn_fwd_lse)
+  * ring-style chunked prefill, B=1, H=16, S_q=4096, S_k=16384, D=128: four
+    KV chunks of 4096 with smooth_k, then merge_state of the four partials
+  * split-KV decode D=128 (H_q=32, H_kv=8) and D=256 (H_q=16, H_kv=4),
+    Lkv=32768, Lq in {1, 4}                                      (attn_splitkv_decode)
+The headline value is prefill-dominated TFLOP/s (algorithmic FLOPs of the
+step / device time); the decode calls are also timed alone as complete
+CUDA-graph-captured operators (microseconds and HBM GB/s), as is merge_state.
+
+L2 (126 MB) is flushed by writing a 512 MB buffer before every timed step and
+every timed replay, outside the timed span.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs the same per-GPU work (independent
+heads / sequences / batches: weak scaling, no data-path collective); rank 0
+prints one JSON line with the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd+LSE TFLOP/s (prefill); split-KV decode µs & HBM GB/s vs B200 peak"
+D128 = 128
+CFG4_SEQ = [512, 1024, 2048, 4096]
+DECODE_SHAPES = [  # (name, Hq, Hkv, D, Lq, Lkv)
+    ("decode_d128_lq1_lkv32768", 32, 8, 128, 1, 32768),
+    ("decode_d128_lq4_lkv32768", 32, 8, 128, 4, 32768),
+    ("decode_d256_lq1_lkv32768", 16, 4, 256, 1, 32768),
+    ("decode_d256_lq4_lkv32768", 16, 4, 256, 4, 32768),
+]
+
+
+def attn_flops(rows_x_keys: int, D: int) -> int:
+    """2*D FLOPs for q.k and 2*D for p*v per (query row, key) pair."""
+    return 4 * D * rows_x_keys
+
+
+FLOPS_CFG4 = attn_flops(24 * sum(s * s for s in CFG4_SEQ), D128)
+FLOPS_CFG5 = attn_flops(16 * 4096 * 16384, D128)
+FLOPS_CFG5_CHUNK = attn_flops(16 * 4096 * 4096, D128)
+
+
+def decode_flops(Hq, D, Lq, Lkv):
+    return attn_flops(Hq * Lq * Lkv, D)
+
+
+def decode_kv_bytes(Hkv, D, Lkv):
+    return 2 * Hkv * Lkv * D * 2
+
+
+MERGE5_BYTES = 4 * 16 * 4096 * (128 * 2 + 4) + 16 * 4096 * (128 * 2 + 4)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.f = None
+
+    def start(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.strip().split(", ") for r in self.f.read().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                for n, val in zip(names, r[5:9]):
+                    if val.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, dist):
+    import torch
+    import split_kv_merge_attn_b200 as skv
+    import workloads as W
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    torch.manual_seed(0)
+    peaks = load_peaks()
+
+    # ---------------- inputs (seeded, generated on the host, copied once)
+    c4 = W.config4(seed=rank)
+    c5 = W.config5(seed=rank)
+    host = {"c4": c4, "c5": c5}
+    q4, k4, v4 = c4["q"].to(dev), c4["k"].to(dev), c4["v"].to(dev)
+    cuq4, cuk4 = c4["cu_seqlens_q"].to(dev), c4["cu_seqlens_k"].to(dev)
+    q5 = c5["q"].to(dev)
+    b5 = c5["chunk_bounds"]
+    k5 = [c5["k"][:, :, a:e].contiguous().to(dev) for a, e in zip(b5[:-1], b5[1:])]
+    v5 = [c5["v"][:, :, a:e].contiguous().to(dev) for a, e in zip(b5[:-1], b5[1:])]
+    dec_in = []
+    for (name, Hq, Hkv, D, Lq, Lkv) in DECODE_SHAPES:
+        if D == 128:
+            d = W.config2(Lq, Lkv, seed=rank)
+        else:
+            d = W.config3(Lq, Lkv, seed=rank)
+        host[name] = d
+        dec_in.append((name, d["q"].to(dev), d["k"].to(dev), d["v"].to(dev), d["scale"]))
+    scale = D128 ** -0.5
+
+    # ---------------- outputs and workspaces
+    out4 = torch.empty_like(q4)
+    lse4 = torch.empty(24, q4.shape[0], dtype=torch.float32, device=dev)
+    ws4 = torch.empty(max(skv.attn_fwd_lse_workspace(4, 24, 24, q4.shape[0], 128, "bf16", "TND", 0), 1),
+                      dtype=torch.uint8, device=dev)
+    o5p = torch.empty((4,) + tuple(q5.shape), dtype=q5.dtype, device=dev)
+    l5p = torch.empty(4, 1, 16, 4096, dtype=torch.float32, device=dev)
+    ws5 = torch.empty(skv.attn_fwd_lse_workspace(1, 16, 16, 4096, 128, "bf16", "HND", 1), dtype=torch.uint8,
+                      device=dev)
+    out5 = torch.empty_like(q5)
+    lse5 = torch.empty(1, 16, 4096, dtype=torch.float32, device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    dec_buf = []
+    for (name, q, k, v, sc) in dec_in:
+        B, Hq, Lq, D = q.shape
+        splits, _ = skv.attn_splitkv_plan(B, Hq, k.shape[1], Lq, k.shape[2], sms, 0)
+        ws = torch.empty(max(skv.attn_splitkv_workspace(B, Hq, Lq, D, splits), 1), dtype=torch.uint8, device=dev)
+        dec_buf.append((torch.empty_like(q), torch.empty(B, Hq, Lq, dtype=torch.float32, device=dev), ws, splits))
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def call_cfg4():
+        skv.attn_fwd_lse(q4, k4, v4, scale, layout="TND", cu_seqlens_q=cuq4, cu_seqlens_k=cuk4,
+                         max_seqlen_q=4096, max_seqlen_k=4096, out=out4, lse=lse4, workspace=ws4)
+
+    def call_cfg5():
+        for c in range(4):
+            skv.attn_fwd_lse(q5, k5[c], v5[c], scale, layout="HND", smooth_k=1, out=o5p[c], lse=l5p[c],
+                             workspace=ws5)
+        skv.merge_state(o5p, l5p, "HND", out=out5, lse=lse5)
+
+    def call_decode(i):
+        name, q, k, v, sc = dec_in[i]
+        o, l, ws, splits = dec_buf[i]
+        skv.attn_splitkv_decode(q, k, v, sc, num_splits=splits, out=o, lse=l, workspace=ws)
+
+    step_flops = FLOPS_CFG4 + FLOPS_CFG5 + sum(decode_flops(Hq, D, Lq, Lkv) for (_, Hq, _, D, Lq, Lkv) in DECODE_SHAPES)
+
+    # events around each call inside the timed step
+    parts = ["cfg4_varlen_prefill", "cfg5_chunked_prefill_merge"] + [s[0] for s in DECODE_SHAPES]
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record()
+        call_cfg4()
+        if evs is not None:
+            evs[1].record()
+        call_cfg5()
+        if evs is not None:
+            evs[2].record()
+        for i in range(len(DECODE_SHAPES)):
+            call_decode(i)
+            if evs is not None:
+                evs[3 + i].record()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert skv.device_error() == 0
+
+    # ---------------- timed region
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.5)
+    n_ev = 3 + len(DECODE_SHAPES)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    launches0 = skv.launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    launches = skv.launch_count() - launches0
+    clocks = sampler.stop() if sampler else None
+    step_ms = [evs[i][0].elapsed_time(evs[i][n_ev - 1]) for i in range(args.steps)]
+    part_ms = {p: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)] for j, p in enumerate(parts)}
+    ms = sum(step_ms) / len(step_ms)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = step_flops * world / (ms * 1e-3) / 1e12
+    assert skv.device_error() == 0
+
+    # ---------------- dominant kernel roofline: the varlen prefill launch
+    pf_us = 1e3 * sum(part_ms["cfg4_varlen_prefill"]) / args.steps
+    pf_tflops = FLOPS_CFG4 / (pf_us * 1e-6) / 1e12
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "prefill_kernel_traffic.json")
+    if os.path.exists(tp):
+        tj = json.load(open(tp))
+        if tj.get("kernel_source_sha256") == kernel_source_hash():
+            traffic = tj.get("dram_bytes_per_launch")
+    roofline = {"bound": "tensor", "achieved": round(pf_tflops, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(pf_tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
+                "kernel": "prefill_kernel<128,bf16> (varlen TND, H=24, seqlens 512..4096)",
+                "peak_source": peaks["source"] + " bf16 burst (kernel timed as one launch)",
+                "launch_us": round(pf_us, 1)}
+
+    # ---------------- per-operation detail (graph-captured decode, merge)
+    detail = {}
+    for p in parts:
+        detail[p] = {"us_in_step": round(1e3 * sum(part_ms[p]) / args.steps, 2)}
+    detail["cfg5_chunked_prefill_merge"]["tflops"] = round(
+        FLOPS_CFG5 / (detail["cfg5_chunked_prefill_merge"]["us_in_step"] * 1e-6) / 1e12, 1)
+    detail["cfg4_varlen_prefill"]["tflops"] = round(pf_tflops, 1)
+
+    def time_graph(fn, reps):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        ts.sort()
+        del g
+        return ts[len(ts) // 2]
+
+    for i, (name, Hq, Hkv, D, Lq, Lkv) in enumerate(DECODE_SHAPES):
+        us = time_graph(lambda i=i: call_decode(i), 50)
+        gbs = decode_kv_bytes(Hkv, D, Lkv) / (us * 1e-6) / 1e9
+        detail[name].update({"graph_us_median": round(us, 2), "kv_gbs": round(gbs, 1),
+                             "hbm_frac": round(gbs / peaks["hbm_gbs"], 3), "splits": dec_buf[i][3]})
+    # merge_state of workload 5 alone (HBM bound)
+    us_m = time_graph(lambda: skv.merge_state(o5p, l5p, "HND", out=out5, lse=lse5), 50)
+    detail["merge_state_cfg5"] = {"graph_us_median": round(us_m, 2),
+                                  "gbs": round(MERGE5_BYTES / (us_m * 1e-6) / 1e9, 1),
+                                  "hbm_frac": round(MERGE5_BYTES / (us_m * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)}
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = run_e2e(args, dev, host, skv, torch, step_flops, world, dist)
+
+    # ---------------- oracle on the host cores (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded randn, workloads/)",
+            "config": {"workload": "one pass over: varlen TND prefill (H24 D128 seqlens 512..4096) + chunked "
+                                   "ring-style prefill with smooth_k (B1 H16 Sq4096 Sk16384 D128, 4 chunks) + "
+                                   "merge_state + split-KV decode (D128 Hq32/Hkv8 and D256 Hq16/Hkv4, Lkv 32768, "
+                                   "Lq 1 and 4)",
+                       "algorithmic_gflop_per_step": round(step_flops / 1e9, 2),
+                       "l2": "flushed (512 MB write) before every timed step and replay",
+                       "parallelism": f"replicas x{world} (independent work per GPU, no exchange)"},
+            "roofline": roofline, "detail": detail, "e2e": e2e, "gpu_launches": int(launches),
+            "clocks": clocks, "cpu_baseline": cpu, "peaks": peaks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, dev, host, skv, torch, step_flops, world, dist):
+    """Same step through the public API, with the step's inputs copied from
+    pinned host memory and its outputs (O and LSE) read back every step."""
+    c4, c5 = host["c4"], host["c5"]
+    pin = lambda t: t.pin_memory()
+    hq4, hk4, hv4 = pin(c4["q"]), pin(c4["k"]), pin(c4["v"])
+    hcu = pin(c4["cu_seqlens_q"])
+    hq5 = pin(c5["q"])
+    b5 = c5["chunk_bounds"]
+    hk5 = [pin(c5["k"][:, :, a:e].contiguous()) for a, e in zip(b5[:-1], b5[1:])]
+    hv5 = [pin(c5["v"][:, :, a:e].contiguous()) for a, e in zip(b5[:-1], b5[1:])]
+    hdec = [(pin(host[n]["q"]), pin(host[n]["k"]), pin(host[n]["v"]), host[n]["scale"]) for (n, *_r) in DECODE_SHAPES]
+    sc = D128 ** -0.5
+    h2d = sum(t.numel() * t.element_size() for t in [hq4, hk4, hv4, hcu, hcu, hq5] + hk5 + hv5)
+    h2d += sum(q.numel() * q.element_size() + k.numel() * k.element_size() * 2 for q, k, v, s in hdec)
+    # outputs read back: O (bf16) and LSE (fp32) of every call
+    d2h_o = [torch.empty_like(hq4, device="cpu").pin_memory(), torch.empty(24, hq4.shape[0]).pin_memory(),
+             torch.empty_like(hq5, device="cpu").pin_memory(), torch.empty(1, 16, 4096).pin_memory()]
+    d2h_o += [torch.empty_like(q, device="cpu").pin_memory() for q, k, v, s in hdec]
+    d2h_o += [torch.empty(q.shape[:3]).pin_memory() for q, k, v, s in hdec]
+    d2h = sum(t.numel() * t.element_size() for t in d2h_o)
+
+    def e2e_step():
+        q4, k4, v4 = hq4.to(dev, non_blocking=True), hk4.to(dev, non_blocking=True), hv4.to(dev, non_blocking=True)
+        cu = hcu.to(dev, non_blocking=True)
+        o4, l4 = skv.attn_fwd_lse(q4, k4, v4, sc, layout="TND", cu_seqlens_q=cu, cu_seqlens_k=cu, max_seqlen_q=4096,
+                                  max_seqlen_k=4096)
+        q5 = hq5.to(dev, non_blocking=True)
+        parts = [skv.attn_fwd_lse(q5, k.to(dev, non_blocking=True), v.to(dev, non_blocking=True), sc, smooth_k=1)
+                 for k, v in zip(hk5, hv5)]
+        o5, l5 = skv.merge_state(torch.stack([p[0] for p in parts]), torch.stack([p[1] for p in parts]))
+        outs = [o4, l4, o5, l5]
+        dec_o, dec_l = [], []
+        for q, k, v, s in hdec:
+            o, l = skv.attn_splitkv_decode(q.to(dev, non_blocking=True), k.to(dev, non_blocking=True),
+                                           v.to(dev, non_blocking=True), s)
+            dec_o.append(o)
+            dec_l.append(l)
+        for dst, src in zip(d2h_o, outs + dec_o + dec_l):
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    n = max(2, min(args.steps, 5))
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(step_flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 3),
+            "steps": n}
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("prefill.cuh", "tcgen05.cuh", "skv_device.cuh"):
+        h.update(open(os.path.join(ROOT, "split_kv_merge_attn_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+# ---------------------------------------------------------------- oracle (CPU)
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(seconds_budget: float):
+    """Runs the oracle on a bounded sample of the step's workload: whole query
+    heads of the chunked workload (all 16384 keys, unsmoothed definition),
+    then query rows of the longest varlen sequence, until the budget is used.
+    Returns (flops, seconds, description)."""
+    import numpy as np
+    import oracle as O
+    import workloads as W
+    c5 = W.config5()
+    q, k, v = (O.to_f64(c5[x])[0] for x in "qkv")
+    flops, t0, heads = 0, time.perf_counter(), 0
+    rows = 512
+    while time.perf_counter() - t0 < seconds_budget and heads < 16:
+        for r0 in range(0, 4096, rows):
+            O.attention_rows(q[heads, r0:r0 + rows], k[heads], v[heads], c5["scale"])
+            flops += attn_flops(rows * 16384, 128)
+            if time.perf_counter() - t0 >= seconds_budget:
+                break
+        heads += 1
+    dt = time.perf_counter() - t0
+    return flops, dt, (f"oracle attention_rows (float64 numpy) on workload-5 query rows in blocks of {rows} "
+                       f"x 16384 keys, D=128: {flops / 1e9:.1f} GFLOP in {dt:.1f} s")
+
+
+def cpu_baseline(budget_s: float = 15.0):
+    flops, dt, desc = oracle_sample(budget_s)
+    return {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": desc}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step is a bounded sample of the
+    same workload on the host cores."""
+    if rank != 0:
+        return
+    per_step = max(2.0, min(20.0, 60.0 / max(args.steps + args.warmup, 1)))
+    for _ in range(args.warmup):
+        oracle_sample(per_step)
+    fl, secs = 0, 0.0
+    desc = ""
+    for _ in range(args.steps):
+        f, dt, desc = oracle_sample(per_step)
+        fl += f
+        secs += dt
+    value = fl / secs / 1e12
+    cores = _blas_threads()
+    line = {"metric": METRIC, "value": round(value, 5), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded randn, workloads/)",
+            "impl": "reference",
+            "config": {"workload": "bounded sample of the same step: workload-5 query rows x all 16384 keys",
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- main
+
+def run_case(args):
+    """Runs one operation of the step `--steps` times with nothing else around
+    it (the small commands the ncu captures use)."""
+    import torch
+    import split_kv_merge_attn_b200 as skv
+    import workloads as W
+    dev = torch.device("cuda", 0)
+    case = args.case
+    if case == "prefill_varlen":
+        c = W.config4()
+        q, k, v = c["q"].to(dev), c["k"].to(dev), c["v"].to(dev)
+        cu = c["cu_seqlens_q"].to(dev)
+        fn = lambda: skv.attn_fwd_lse(q, k, v, c["scale"], layout="TND", cu_seqlens_q=cu, cu_seqlens_k=cu,
+                                      max_seqlen_q=4096, max_seqlen_k=4096)
+    elif case == "prefill_chunk":
+        c = W.config5(Sk=4096, n_chunks=1)
+        q, k, v = c["q"].to(dev), c["k"].to(dev), c["v"].to(dev)
+        fn = lambda: skv.attn_fwd_lse(q, k, v, c["scale"], smooth_k=1)
+    elif case.startswith("decode_"):
+        name = [s for s in DECODE_SHAPES if s[0] == case][0]
+        _, Hq, Hkv, D, Lq, Lkv = name
+        d = W.config2(Lq, Lkv) if D == 128 else W.config3(Lq, Lkv)
+        q, k, v = d["q"].to(dev), d["k"].to(dev), d["v"].to(dev)
+        fn = lambda: skv.attn_splitkv_decode(q, k, v, d["scale"])
+    elif case == "merge5":
+        g = torch.Generator().manual_seed(0)
+        o = torch.randn(4, 1, 16, 4096, 128, generator=g).bfloat16().to(dev)
+        l = (torch.randn(4, 1, 16, 4096, generator=g) * 10).to(dev)
+        fn = lambda: skv.merge_state(o, l)
+    else:
+        raise SystemExit(f"unknown case {case}")
+    for _ in range(args.steps):
+        fn()
+    torch.cuda.synchronize()
+    assert skv.device_error() == 0
+    print(json.dumps({"case": case, "runs": args.steps, "ok": True}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None, help="run one operation only (for profiler captures)")
+    args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -93,19 +93,28 @@ typedef enum { SKV_HND = 0, SKV_NHD = 1, SKV_TND = 2 } skv_layout;
  *   (used to size the grid); max_seqlen_k is accepted for API symmetry.
  * Non-causal: every query row sees every key of its sequence.
  *
- * smooth_k != 0: before the product, K is replaced by K' = K - mean(K) with the
- * mean taken in fp32 over the call's own KV range, per (batch or sequence,
- * kv head, channel), rounded back to the input type; the LSE is corrected by
- * adding scale * (q_i . mean(K)) / ln 2, so it stays the LSE of the ORIGINAL
- * logits (ARK issue, second issue and part 3 of the repro).  O is unchanged up
- * to rounding (softmax is shift invariant).  Needs workspace (see below).
+ * smooth_k (ARK issue, second issue and part 3 of the repro): K is smoothed by
+ * its mean mu over the call's own KV range, taken in fp32 per (batch or
+ * sequence, kv head, channel), and the LSE is corrected by adding
+ * scale * (q_i . mu) / ln 2 so that it stays the LSE of the ORIGINAL logits --
+ * partial LSEs of chunks with different means then lie on one scale.  O is
+ * unchanged up to rounding (softmax is shift invariant).
+ *   0: no smoothing.
+ *   1: the smoothing is applied to the fp32 logits, s_ij - scale * q_i . mu,
+ *      which is exactly K' = K - mu with no 16-bit rounding of K'.
+ *   2: K' = K - mu is materialised in the input type in the workspace and used
+ *      by the tensor cores; the rounding of K' to 16 bits perturbs the logits
+ *      by about scale * |q| * 2^-9 * |K'| (the LSE is then accurate to that).
+ *   Both modes need workspace (see below); for varlen, max_seqlen_k must bound
+ *   every key length.
  *
- * scale: the logit scale (e.g. D^-0.5), finite.
+ * scale: the logit scale (e.g. D^-0.5), finite and > 0.
+ * k and v may be NULL only when there are no keys (Sk == 0).
  * workspace: device, >= attn_fwd_lse_workspace(...) bytes, 256-byte aligned;
  *   may be NULL when that query returns 0.  After a varlen call its first
  *   bytes hold the work order: int32 order[B] (sequences, longest kv first,
  *   ties by index) then int32 offsets[B+1] (prefix sums of Hq*ceil(len_q/256)).
- * Errors: SKV_ERR_INVALID_ARG for NULL q/k/v/out, non-positive sizes (B, Hq,
+ * Errors: SKV_ERR_INVALID_ARG for NULL q/out, NULL k/v with keys, non-positive sizes (B, Hq,
  *   Hkv, D; Sq, Sk may be 0 in the dense case), Hq % Hkv != 0, misaligned
  *   pointers, unknown layout/dtype, or missing/extra cu_seqlens;
  *   SKV_ERR_UNSUPPORTED for D not in {64,128} or dtype fp32.
@@ -207,6 +216,10 @@ int skv_last_cuda_error(void);
  * outputs are undefined).  Synchronises the device.  Returns SKV_ERR_CUDA if the
  * read itself fails. */
 skv_status skv_device_error(int* code);
+
+/* Number of kernels this library has launched in this process so far (all
+ * devices, all threads).  Benchmarks difference it around a timed region. */
+uint64_t skv_launch_count(void);
 
 /* Library version, e.g. "0.1.0". */
 const char* skv_version(void);

@@ -45,6 +45,7 @@ SIGNATURES = {
     "skv_last_cuda_error": (_c_int, []),
     "skv_device_error": (_c_int, [_vp]),
     "skv_version": (ctypes.c_char_p, []),
+    "skv_launch_count": (ctypes.c_uint64, []),
 }
 
 _lib = None
@@ -159,6 +160,11 @@ def attn_varlen_plan(cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int], H
     offsets = (ctypes.c_int32 * (B + 1))()
     _check(lib().attn_varlen_plan(cq, ck, B, Hq, order, offsets), "attn_varlen_plan")
     return list(order)[:B], list(offsets)
+
+
+def launch_count() -> int:
+    """Kernels launched by the library in this process so far."""
+    return int(lib().skv_launch_count())
 
 
 def device_error() -> int:
@@ -283,5 +289,5 @@ def merge_state(o_parts, lse_parts, layout: str = "HND", out=None, lse=None, out
 
 
 __all__ = ["attn_fwd_lse", "attn_splitkv_decode", "merge_state", "attn_splitkv_plan", "attn_splitkv_workspace",
-           "attn_fwd_lse_workspace", "attn_varlen_plan", "device_error", "lib", "SkvError", "status_string",
+           "attn_fwd_lse_workspace", "attn_varlen_plan", "device_error", "launch_count", "lib", "SkvError", "status_string",
            "LIB_PATH", "SIGNATURES"]

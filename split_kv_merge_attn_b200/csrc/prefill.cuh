@@ -66,6 +66,8 @@ struct PrefillArgs {
   void* out;
   float* lse;
   const float* kmean;   // smooth: [Bseq, Hkv, D] fp32, else null
+  int shift_logits;     // smooth: 1 = subtract the mean term from the fp32 logits (K unsmoothed),
+                        //         0 = K was replaced by K' = K - mean (already smoothed)
   const int* cu_q;
   const int* cu_k;
   const int* order;
@@ -336,6 +338,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
       }
 
+      // logits seen by the softmax are the smoothed ones: K' = K - mean either
+      // materialised (K' in the MMA) or applied here as a per-row fp32 shift
+      const float bias_shift = a.shift_logits ? delta : 0.f;
       float m_run = -INFINITY;  // running max of the (smoothed) log2-domain logits, possibly stale
       float l_run = 0.f;
       for (int j = 0; j < nkv && ok; ++j) {
@@ -358,7 +363,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         float mx = s[0];
 #pragma unroll
         for (int c = 1; c < kPfBN; ++c) mx = fmaxf(mx, s[c]);
-        const float t_max = fmaf(mx, a.scale_log2, -delta);
+        const float t_max = fmaf(mx, a.scale_log2, -bias_shift);
         const float m_new = fmaxf(m_run, t_max);
         const bool rescale = m_new > m_run + kPfRescaleThreshold;
         float alpha = 1.f;
@@ -367,7 +372,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           m_run = m_new;
         }
         l_run *= alpha;
-        const float neg_bias = -(m_run + delta);
+        const float neg_bias = -(m_run + bias_shift);
         float psum = 0.f;
 #pragma unroll
         for (int c = 0; c < kPfBN / 32; ++c) {

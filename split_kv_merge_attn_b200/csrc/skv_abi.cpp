@@ -81,6 +81,8 @@ int skv_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char* skv_version(void) { return "0.1.0"; }
 
+uint64_t skv_launch_count(void) { return skv::launch_count(); }
+
 skv_status skv_device_error(int* code) {
   if (code == nullptr) return SKV_ERR_INVALID_ARG;
   return cuda_status(skv::read_and_clear_device_error(code));
@@ -231,6 +233,7 @@ skv_status attn_fwd_lse(const void* q, const void* k, const void* v, void* out, 
                                  D, dtype, layout, stream);
     if (e) return cuda_status(e);
     p.kmean = kmean;
+    p.shift_logits = smooth_k == 1 ? 1 : 0;
     if (smooth_k == 2) p.k = kprime;
   }
   return cuda_status(skv::launch_prefill(p, stream));

@@ -47,6 +47,7 @@ struct PrefillLaunch {
   void* out;
   float* lse;
   const float* kmean;      // [B(or seqs), Hkv, D] fp32 when smooth_k, else null
+  int shift_logits;        // smooth_k == 1: apply the mean shift to the logits
   const int32_t* cu_q;     // device, varlen only
   const int32_t* cu_k;
   const int32_t* order;    // device work order (varlen)
@@ -69,5 +70,9 @@ int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partia
                     int Hkv, int Sk, int max_len, int D, skv_dtype dt, skv_layout layout, skv_stream_t stream);
 
 int read_and_clear_device_error(int* code);
+
+// Launch accounting (incremented by every successful kernel launch).
+void count_launches(int n);
+uint64_t launch_count();
 
 }  // namespace skv

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -29,6 +30,18 @@ int read_and_clear_device_error(int* code) {
   *code = v;
   return 0;
 }
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+// returns e unchanged; counts n launches when e reports success
+int counted(int e, int n) {
+  if (e == 0) g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed);
+  return e;
+}
+}  // namespace
+
+void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+uint64_t launch_count() { return g_launches.load(std::memory_order_relaxed); }
 
 // ------------------------------------------------------------ device info
 
@@ -130,7 +143,7 @@ int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, f
   else if (parts_dt == SKV_FP16 && out_dt == SKV_BF16) SKV_MERGE(__half, __nv_bfloat16);
   else return cudaErrorInvalidValue;
 #undef SKV_MERGE
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 // ------------------------------------------------------------ decode
@@ -144,7 +157,7 @@ int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeAr
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kDecodeThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 }  // namespace
 
@@ -223,7 +236,7 @@ int launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kPfThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, a);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 }  // namespace
 
@@ -245,6 +258,7 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   a.out = p.out;
   a.lse = p.lse;
   a.kmean = p.kmean;
+  a.shift_logits = p.shift_logits;
   a.cu_q = p.cu_q;
   a.cu_k = p.cu_k;
   a.order = p.order;
@@ -281,7 +295,7 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
 int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int32_t* order, int32_t* offsets,
                        skv_stream_t stream) {
   varlen_plan_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(cu_q, cu_k, B, Hq, order, offsets);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 // ------------------------------------------------------------ smooth_k
@@ -312,7 +326,8 @@ int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partia
     if (dt == SKV_BF16) ksmooth_write_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
     else ksmooth_write_kernel<__half><<<grid, 256, 0, st>>>(a);
   }
-  return cudaGetLastError();
+  const int n = 1 + (a.nchunks > 0 ? 1 : 0) + (k_smoothed != nullptr && a.nchunks > 0 ? 1 : 0);
+  return counted(cudaGetLastError(), n);
 }
 
 }  // namespace skv
