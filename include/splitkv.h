@@ -166,12 +166,13 @@ skv_status attn_splitkv_decode(const void* q, const void* k, const void* v, void
 /* Split plan (host, pure integer).  For n keys, split s covers
  *   [s*C, min((s+1)*C, n)),  C = 64 * ceil(ceil(n / num_splits) / 64).
  * If requested_splits > 0 it is used as is (1..256); otherwise the count is
- * chosen to give every one of num_sms SMs two CTAs (CTAs = B * Hkv *
- * ceil(G*Lq/16) * splits, G = Hq/Hkv), keeping >= 128 keys per split, at most
- * 256 splits, and none that the rounding of C would leave empty.
+ * chosen so the decode grid fills num_splits SMs: B * Hkv * ceil(G*Lq/16) *
+ * splits CTAs (G = Hq/Hkv) aiming at two CTAs per SM for D <= 128 and one for
+ * D = 256 (the kernel's residency), keeping >= 128 keys per split, at most 256
+ * splits, and none that the rounding of C would leave empty.
  * Writes *num_splits and, if bounds != NULL, bounds[0..num_splits] (host) with
  * split s = [bounds[s], bounds[s+1]). */
-skv_status attn_splitkv_plan(int B, int Hq, int Hkv, int Lq, int n, int num_sms,
+skv_status attn_splitkv_plan(int B, int Hq, int Hkv, int Lq, int n, int D, int num_sms,
                              int requested_splits, int* num_splits, int32_t* bounds);
 
 /* Workspace bytes for a decode with this many splits (fp32 partial O and LSE). */

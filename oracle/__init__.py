@@ -253,7 +253,8 @@ def lse_varlen_to_dense(lse_ht: np.ndarray, B: int, S: int) -> np.ndarray:
 SPLIT_ALIGN = 64          # split chunk is a multiple of this many keys
 SPLIT_MIN_KEYS = 128      # the automatic plan keeps at least this many keys per split
 SPLIT_MAX = 256           # upper limit on the number of splits
-CTAS_PER_SM = 2           # the automatic plan aims for this many CTAs per SM
+CTAS_PER_SM = 2           # the automatic plan aims for this many CTAs per SM (D <= 128) ...
+CTAS_PER_SM_D256 = 1      # ... and this many for D = 256 (one decode CTA fills an SM)
 DECODE_ROWS_PER_CTA = 16  # query rows (G * Lq) one decode CTA handles
 PREFILL_ROWS_PER_CTA = 256
 
@@ -277,14 +278,15 @@ def split_bounds(n: int, num_splits: int) -> List[int]:
     return [min(s * C, n) for s in range(num_splits + 1)]
 
 
-def auto_num_splits(B: int, Hkv: int, Hq: int, Lq: int, n: int, num_sms: int) -> int:
-    """Automatic split count: enough CTAs to give every SM CTAS_PER_SM of them,
-    no split shorter than SPLIT_MIN_KEYS keys, at most SPLIT_MAX, and no
-    split that the chunk rounding would leave empty."""
+def auto_num_splits(B: int, Hkv: int, Hq: int, Lq: int, n: int, num_sms: int, D: int = 128) -> int:
+    """Automatic split count: enough CTAs to give every SM CTAS_PER_SM of them
+    (CTAS_PER_SM_D256 for D = 256), no split shorter than SPLIT_MIN_KEYS keys,
+    at most SPLIT_MAX, and no split that the chunk rounding would leave empty.
+    (Reading of "num_splits sized to fill the SMs": the pages give no formula.)"""
     G = Hq // Hkv
     row_groups = _ceil_div(G * Lq, DECODE_ROWS_PER_CTA)
     units = B * Hkv * row_groups
-    target = CTAS_PER_SM * num_sms
+    target = (CTAS_PER_SM_D256 if D > 128 else CTAS_PER_SM) * num_sms
     s = max(1, _ceil_div(target, max(units, 1)))
     s = min(s, max(1, _ceil_div(n, SPLIT_MIN_KEYS)), SPLIT_MAX)
     if n > 0:

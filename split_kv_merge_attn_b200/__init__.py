@@ -37,7 +37,7 @@ SIGNATURES = {
     "attn_varlen_plan": (_c_int, [_vp, _vp, _c_int, _c_int, _vp, _vp]),
     "attn_splitkv_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_float, _c_int, _vp, _c_int, _vp, _c_size, _vp]),
-    "attn_splitkv_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
+    "attn_splitkv_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "attn_splitkv_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "merge_state": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                              _c_i64, _c_i64, _vp]),
@@ -130,14 +130,14 @@ def _workspace(nbytes: int, device, workspace):
 
 # ------------------------------------------------------------------ queries
 
-def attn_splitkv_plan(B: int, Hq: int, Hkv: int, Lq: int, n: int, num_sms: int = 148,
+def attn_splitkv_plan(B: int, Hq: int, Hkv: int, Lq: int, n: int, D: int = 128, num_sms: int = 148,
                       requested_splits: int = 0) -> Tuple[int, list]:
     """Host split plan: (num_splits, bounds[num_splits + 1])."""
     ns = ctypes.c_int(0)
-    _check(lib().attn_splitkv_plan(B, Hq, Hkv, Lq, n, num_sms, requested_splits, ctypes.byref(ns), None),
+    _check(lib().attn_splitkv_plan(B, Hq, Hkv, Lq, n, D, num_sms, requested_splits, ctypes.byref(ns), None),
            "attn_splitkv_plan")
     bounds = (ctypes.c_int32 * (ns.value + 1))()
-    _check(lib().attn_splitkv_plan(B, Hq, Hkv, Lq, n, num_sms, requested_splits, ctypes.byref(ns), bounds),
+    _check(lib().attn_splitkv_plan(B, Hq, Hkv, Lq, n, D, num_sms, requested_splits, ctypes.byref(ns), bounds),
            "attn_splitkv_plan")
     return ns.value, list(bounds)
 
@@ -250,7 +250,7 @@ def attn_splitkv_decode(q, k, v, scale: Optional[float] = None, kv_len=None, num
     splits = num_splits
     if splits == 0:
         sms = torch.cuda.get_device_properties(q.device).multi_processor_count
-        splits, _ = attn_splitkv_plan(B, Hq, Hkv, Lq, Lkv, sms, 0)
+        splits, _ = attn_splitkv_plan(B, Hq, Hkv, Lq, Lkv, D, sms, 0)
     nbytes = attn_splitkv_workspace(B, Hq, Lq, D, splits)
     workspace, wbytes = _workspace(nbytes, q.device, workspace)
     st = lib().attn_splitkv_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lkv, D,

@@ -119,6 +119,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
     }
   }
   __syncthreads();
+  // let a programmatically dependent merge launch be scheduled; it still waits
+  // for this whole grid to finish before it reads the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int64_t row0 = (static_cast<int64_t>(b) * a.Hkv + hkv) * a.Lkv;
 

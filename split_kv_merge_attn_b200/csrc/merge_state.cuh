@@ -134,4 +134,93 @@ __global__ void __launch_bounds__(256) merge_state_kernel(MergeArgs a) {
   }
 }
 
+// Variant for few rows and many parts (the cross-split reduce of a decode:
+// tens of rows, tens of splits).  One CTA per row; its 256 threads split into
+// (D/8) column slices x (256 / (D/8)) part lanes.  Each thread issues the
+// loads of all its parts (LSE and O slice) at once and merges them with a
+// running max of its own; the part lanes are then rescaled to the row max and
+// summed through shared memory -- one round trip to memory instead of one per
+// part.  A part of LSE -inf contributes nothing (its O slot is never used in
+// arithmetic).  Launched as a programmatic dependent of the split kernel, it
+// waits for that grid's results with griddepcontrol.wait.
+template <typename TI, typename TO>
+__global__ void __launch_bounds__(256) merge_state_parts_kernel(MergeArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const TI* __restrict__ op = static_cast<const TI*>(a.o_parts);
+  const float* __restrict__ lp = a.lse_parts;
+  TO* __restrict__ out = static_cast<TO*>(a.out);
+  const int vpr = a.D >> 3;
+  const int lanes = 256 / vpr;
+  const int c = threadIdx.x % vpr;
+  const int pl = threadIdx.x / vpr;
+  const int64_t row = blockIdx.x;
+  int64_t lrow = row;
+  if (a.layout_bsh) {
+    const int h = static_cast<int>(row % a.H);
+    const int64_t bs = row / a.H;
+    const int s = static_cast<int>(bs % a.S);
+    const int64_t b = bs / a.S;
+    lrow = (b * a.H + h) * a.S + s;
+  }
+  __shared__ float red[256 * 8];
+  __shared__ float wmax[8];
+  __shared__ float wsum[256];
+  float m = -INFINITY, W = 0.f;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const TI* base = op + row * a.D + c * 8;
+  constexpr int R = 4;
+  if (pl < lanes) {
+    for (int p0 = pl; p0 < a.P; p0 += R * lanes) {
+      float L[R];
+      float x[R][8];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {  // every load of this batch is issued before any use
+        const int p = p0 + r * lanes;
+        L[r] = (p < a.P) ? __ldg(lp + p * a.part_stride_lse + lrow) : -INFINITY;
+        if (p < a.P) Vec8<TI>::load(base + p * a.part_stride_o, x[r]);
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (L[r] == -INFINITY) continue;
+        const float mn = fmaxf(m, L[r]);
+        const float sc = exp2f(m - mn);  // 0 while m is -inf
+        const float w = exp2f(L[r] - mn);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, x[r][e], acc[e] * sc);
+        W = W * sc + w;
+        m = mn;
+      }
+    }
+  }
+  // row max over all threads
+  float M = m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = M;
+  __syncthreads();
+  M = wmax[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) M = fmaxf(M, wmax[w]);
+  const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[threadIdx.x * 8 + e] = acc[e] * f;
+  wsum[threadIdx.x] = (c == 0) ? W * f : 0.f;
+  __syncthreads();
+  if (pl == 0) {
+    float Wt = 0.f;
+    for (int l = 0; l < lanes; ++l) Wt += wsum[l * vpr];
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = 0.f;
+    for (int l = 0; l < lanes; ++l)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] += red[(l * vpr + c) * 8 + e];
+    const float inv = (M != -INFINITY && Wt > 0.f) ? 1.0f / Wt : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] *= inv;
+    Vec8<TO>::store(out + row * a.D + c * 8, v);
+    if (c == 0 && a.lse != nullptr) a.lse[lrow] = (M == -INFINITY) ? -INFINITY : M + log2f(Wt);
+  }
+}
+
 }  // namespace skv

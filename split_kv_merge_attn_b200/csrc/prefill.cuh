@@ -18,11 +18,9 @@
 // packed 16-bit pairs into S_a's first 64 columns, and O_a += P_a V_j reads P_a
 // straight from TMEM (A operand in tensor memory).
 //
-// Per KV tile j the MMA thread issues PV_0(j), PV_1(j), then S_0(j+1),
-// S_1(j+1).  The next S into S_a overwrites P_a, which PV_a(j) reads; the PTX
-// ISA orders consecutive MMAs only when they share an accumulator, so the MMA
-// thread waits for PV_a(j) to complete (its own commit barrier) before issuing
-// S_a(j+1); the other tile's MMA keeps the tensor pipe busy meanwhile.
+// The MMA thread alternates between the tiles (S_0(j), PV_1(j-1), S_1(j),
+// PV_0(j)), so while the softmax warps of one tile exponentiate, the tensor
+// core works on the other tile.
 //
 // Online softmax in the exp2 domain with a lazily updated running max: the
 // max is only raised (and O_a rescaled in TMEM) when it grows by more than 8
@@ -43,19 +41,80 @@ constexpr int kPfBN = 128;          // keys per KV tile
 constexpr int kPfThreads = 320;
 constexpr float kPfRescaleThreshold = 8.0f;
 
+// Tuning switches (compile time).  SKV_PF_ONEPASS: S is read from TMEM once
+// (128 registers of logits per thread) instead of twice in halves.
+// SKV_PF_POLY_PAIRS: of every 16 pairs of probabilities, this many are
+// computed with the FMA-pipe polynomial below instead of the MUFU ex2.
+#ifndef SKV_PF_ONEPASS
+#define SKV_PF_ONEPASS 0
+#endif
+#ifndef SKV_PF_POLY_PAIRS
+#define SKV_PF_POLY_PAIRS 0
+#endif
+
+// 2^x on the FMA pipe for x in [-126, 2^22): Cody-Waite style split
+// x = n + r with n = round(x) (the 1.5 * 2^23 addition trick) and r in
+// [-1/2, 1/2], 2^r from a degree-3 polynomial fitted to minimise the maximum
+// relative error on [-1/2, 1/2] (7.5e-5; coefficients from exp2_poly_fit.py
+// beside this file), and 2^n applied by adding n to the exponent field.
+// Arguments below -126 are clamped there (result < 2^-125, i.e. 0 for every
+// sum it enters).  Used for a fraction of the softmax probabilities so the
+// MUFU exp unit is not the only one working.
+constexpr float kExp2C0 = 0.9999280729428965f;
+constexpr float kExp2C1 = 0.6932609762204822f;
+constexpr float kExp2C2 = 0.2426111270828907f;
+constexpr float kExp2C3 = 0.05517171959872975f;
+
+__device__ __forceinline__ void poly_exp2_pair(uint64_t x2, float& p0, float& p1) {
+  float2 x = f2_unpack(x2);
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const uint64_t xc = f2_pack(x.x, x.y);
+  const uint64_t y = fadd2(xc, f2_pack(12582912.f, 12582912.f));    // round(x) in the low mantissa bits
+  const uint64_t n = fadd2(y, f2_pack(-12582912.f, -12582912.f));   // round(x) as a float
+  const uint64_t r = ffma2(n, f2_pack(-1.f, -1.f), xc);              // x - round(x), exact
+  uint64_t q = ffma2(f2_pack(kExp2C3, kExp2C3), r, f2_pack(kExp2C2, kExp2C2));
+  q = ffma2(q, r, f2_pack(kExp2C1, kExp2C1));
+  q = ffma2(q, r, f2_pack(kExp2C0, kExp2C0));
+  const float2 qf = f2_unpack(q), yf = f2_unpack(y);
+  p0 = __uint_as_float(__float_as_uint(qf.x) + (__float_as_uint(yf.x) << 23));
+  p1 = __uint_as_float(__float_as_uint(qf.y) + (__float_as_uint(yf.y) << 23));
+}
+
+// Exponentiates 64 logits (32 pairs) of one row: p = 2^(s * scale_log2 + nb),
+// packs them as 16-bit pairs and accumulates the row sum in packed fp32 pairs.
+template <bool kPoly, typename T>
+__device__ __forceinline__ void exp_pack_64(const float (&sv)[64], uint64_t sc2, uint64_t nb2, uint32_t (&pk)[32],
+                                            uint64_t (&ps2)[2]) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const uint64_t x2 = ffma2(f2_pack(sv[2 * e], sv[2 * e + 1]), sc2, nb2);
+    float p0, p1;
+    if (kPoly && ((e % 16) * SKV_PF_POLY_PAIRS) % 16 < SKV_PF_POLY_PAIRS) {
+      poly_exp2_pair(x2, p0, p1);
+    } else {
+      const float2 x = f2_unpack(x2);
+      p0 = ex2_approx(x.x);
+      p1 = ex2_approx(x.y);
+    }
+    ps2[e & 1] = fadd2(ps2[e & 1], f2_pack(p0, p1));
+    pk[e] = pack2<T>(p0, p1);
+  }
+}
+
 template <int D>
 struct PrefillCfg {
   static constexpr int kBoxes = D / 64;
   static constexpr int kBoxBytes = 128 * 128;       // 128 rows x 128 bytes
   static constexpr int kQTileBytes = kBoxes * kBoxBytes;
   static constexpr int kKVTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kStages = (D == 64) ? 8 : 4;
+  static constexpr int kStages = (D == 64) ? 8 : 5;
   static constexpr int kRingBytes = kStages * kKVTileBytes;
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = 2 * kQTileBytes;
   static constexpr int kOffBar = kOffRing + kRingBytes;
-  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], pv_done[2], o_full[2], drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 * 4 + 1;
+  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_half[2][2], o_full[2], drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + TMEM slot, abort flag; + alignment pad
   static constexpr int kSCol0 = 0, kSCol1 = 128, kOCol0 = 256, kOCol1 = 256 + D;
@@ -94,9 +153,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + Cfg::kStages;
   uint64_t* s_full = kv_empty + Cfg::kStages;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 2;
-  uint64_t* o_full = pv_done + 2;
+  uint64_t* p_half = s_full + 2;     // [tile][half]: P columns of keys [64h, 64h+64) are in TMEM
+  uint64_t* o_full = p_half + 4;
   uint64_t* drain = o_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 8);
@@ -169,7 +227,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   // ---------------- setup
   if (tid == 0) {
-    for (int i = 0; i < Cfg::kNumBars; ++i) mbar_init(&bars[i], (&bars[i] == &p_full[0] || &bars[i] == &p_full[1]) ? 128u : 1u);
+    for (int i = 0; i < Cfg::kNumBars; ++i) {
+      const bool per_thread = &bars[i] >= &p_half[0] && &bars[i] < &p_half[4];
+      mbar_init(&bars[i], per_thread ? 128u : 1u);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -233,67 +294,93 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
   } else if (warp == 9) {
     // ======================= MMA issuer
+    // Issue order (ping-pong between the two query tiles, so their softmax
+    // phases alternate on the exp units):
+    //   S_0(0) S_1(0) PV_0(0) | S_0(j) PV_1(j-1) S_1(j) PV_0(j) | PV_1(last)
+    // S_t(j) overwrites the TMEM columns that PV_t(j-1) reads P_t from; the two
+    // are issued back to back by this one thread and executed in issue order,
+    // the ordering NVIDIA's CUTLASS Blackwell FMHA also relies on.
     if (lane == 0) {
-      const uint32_t q_addr[2] = {smem_u32(qtile[0]), smem_u32(qtile[1])};
       const uint32_t ring_addr = smem_u32(ring);
-      const uint32_t s_col[2] = {tmem + Cfg::kSCol0, tmem + Cfg::kSCol1};
-      const uint32_t o_col[2] = {tmem + Cfg::kOCol0, tmem + Cfg::kOCol1};
-      bool ok = mbar_wait(q_full, 0, abort_flag, kErrPrefillWait);
-      auto issue_s = [&](int t, uint32_t kaddr) {
+      const uint32_t q0 = smem_u32(qtile[0]), q1 = smem_u32(qtile[1]);
+      const uint32_t s0c = tmem + Cfg::kSCol0, s1c = tmem + Cfg::kSCol1;
+      const uint32_t o0c = tmem + Cfg::kOCol0, o1c = tmem + Cfg::kOCol1;
+      // Shared-memory descriptors are built once; every MMA then only adds a
+      // constant to the start-address field (shared addresses are < 256 KB, so
+      // the 14-bit field never carries).  This keeps the issuing thread cheap:
+      // it shares its scheduler with two softmax warps.
+      const uint64_t dq0 = tc5::smem_desc(q0, 16, 1024), dq1 = tc5::smem_desc(q1, 16, 1024);
+      const uint64_t dk_base = tc5::smem_desc(ring_addr, 16, 1024);
+      const uint64_t dv_base = tc5::smem_desc(ring_addr, Cfg::kBoxBytes, 1024);
+      auto issue_s = [&](uint64_t dq, uint32_t sc, int u) {
+        const uint64_t dk = dk_base + static_cast<uint64_t>(((u % Cfg::kStages) * Cfg::kKVTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Cfg::kBoxBytes + (kk & 3) * 32;
-          tc5::mma_ss(s_col[t], tc5::smem_desc(q_addr[t] + off, 16, 1024), tc5::smem_desc(kaddr + off, 16, 1024),
-                      kIdescQK, kk > 0 ? 1u : 0u);
+          const uint64_t o = static_cast<uint64_t>(((kk >> 2) * Cfg::kBoxBytes + (kk & 3) * 32) >> 4);
+          tc5::mma_ss(sc, dq + o, dk + o, kIdescQK, kk > 0 ? 1u : 0u);
         }
       };
-      if (ok) {
-        const int buf0 = 0;
-        ok = mbar_wait(&kv_full[buf0], 0, abort_flag, kErrPrefillWait);
-        if (ok) {
-          tc5::fence_after();
-          for (int t = 0; t < nt; ++t) {
-            issue_s(t, ring_addr + buf0 * Cfg::kKVTileBytes);
-            tc5::commit(smem_u32(&s_full[t]));
-          }
-          tc5::commit(smem_u32(&kv_empty[buf0]));
-        }
-      }
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int uv = 2 * j + 1;
-        const int bufv = uv % Cfg::kStages;
-        if (!mbar_wait(&kv_full[bufv], (uv / Cfg::kStages) & 1, abort_flag, kErrPrefillWait)) { ok = false; break; }
-        const uint32_t vaddr = ring_addr + bufv * Cfg::kKVTileBytes;
-        for (int t = 0; t < nt; ++t) {
-          if (!mbar_wait(&p_full[t], j & 1, abort_flag, kErrPrefillWait)) { ok = false; break; }
-          tc5::fence_after();
+      auto issue_pv_half = [&](uint32_t sc, uint32_t oc, int u, bool acc, int hf) {
+        const uint64_t dv = dv_base + static_cast<uint64_t>(((u % Cfg::kStages) * Cfg::kKVTileBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kPfBN / 16; ++kk) {
-            tc5::mma_ts(o_col[t], s_col[t] + kk * 8, tc5::smem_desc(vaddr + kk * 2048, Cfg::kBoxBytes, 1024),
-                        kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc5::commit(smem_u32(&pv_done[t]));
+        for (int k4 = 0; k4 < kPfBN / 32; ++k4) {
+          const int kk = hf * (kPfBN / 32) + k4;
+          tc5::mma_ts(oc, sc + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
+                      (acc || kk > 0) ? 1u : 0u);
         }
-        if (!ok) break;
-        tc5::commit(smem_u32(&kv_empty[bufv]));
-        if (j + 1 < nkv) {
-          const int uk = 2 * (j + 1);
-          const int bufk = uk % Cfg::kStages;
-          if (!mbar_wait(&kv_full[bufk], (uk / Cfg::kStages) & 1, abort_flag, kErrPrefillWait)) { ok = false; break; }
-          tc5::fence_after();
-          for (int t = 0; t < nt; ++t) {
-            // P_t(j) lives in S_t's columns: PV_t(j) must finish reading it first
-            if (!mbar_wait(&pv_done[t], j & 1, abort_flag, kErrPrefillWait)) { ok = false; break; }
-            tc5::fence_after();
-            issue_s(t, ring_addr + bufk * Cfg::kKVTileBytes);
-            tc5::commit(smem_u32(&s_full[t]));
-          }
-          if (!ok) break;
-          tc5::commit(smem_u32(&kv_empty[bufk]));
-        } else {
-          for (int t = 0; t < nt; ++t) tc5::commit(smem_u32(&o_full[t]));
+      };
+      auto wait_kv = [&](int u) -> bool {
+        const bool r = mbar_wait(&kv_full[u % Cfg::kStages], (u / Cfg::kStages) & 1, abort_flag, kErrPrefillWait);
+        tc5::fence_after();
+        return r;
+      };
+      auto wait_p = [&](int t, int hf, int j) -> bool {
+        const bool r = mbar_wait(&p_half[2 * t + hf], j & 1, abort_flag, kErrPrefillWait);
+        tc5::fence_after();
+        return r;
+      };
+      // PV of tile t for KV tile j, started on the first 64 keys of P while the
+      // softmax still exponentiates the second 64
+      auto issue_pv = [&](int t, int u, bool acc, int j) -> bool {
+        const uint32_t sc = t ? s1c : s0c, oc = t ? o1c : o0c;
+        if (!wait_p(t, 0, j)) return false;
+        issue_pv_half(sc, oc, u, acc, 0);
+        if (!wait_p(t, 1, j)) return false;
+        issue_pv_half(sc, oc, u, acc, 1);
+        return true;
+      };
+      auto release = [&](int u) { tc5::commit(smem_u32(&kv_empty[u % Cfg::kStages])); };
+      const bool two = nt == 2;
+
+      bool ok = mbar_wait(q_full, 0, abort_flag, kErrPrefillWait) && wait_kv(0);
+      if (ok) {
+        issue_s(dq0, s0c, 0);
+        tc5::commit(smem_u32(&s_full[0]));
+        if (two) {
+          issue_s(dq1, s1c, 0);
+          tc5::commit(smem_u32(&s_full[1]));
         }
+        release(0);
+        ok = wait_kv(1) && issue_pv(0, 1, false, 0);
+        if (ok && nkv == 1) tc5::commit(smem_u32(&o_full[0]));
       }
+      for (int j = 1; j < nkv && ok; ++j) {
+        const int uk = 2 * j, uv = 2 * j + 1;
+        if (!wait_kv(uk)) { ok = false; break; }
+        issue_s(dq0, s0c, uk);
+        tc5::commit(smem_u32(&s_full[0]));
+        if (two && !issue_pv(1, uv - 2, j - 1 > 0, j - 1)) { ok = false; break; }
+        release(uv - 2);              // V_{j-1}: both of its PV products are issued
+        if (two) {
+          issue_s(dq1, s1c, uk);
+          tc5::commit(smem_u32(&s_full[1]));
+        }
+        release(uk);                  // K_j: both S products are issued
+        if (!wait_kv(uv)) { ok = false; break; }
+        if (!issue_pv(0, uv, true, j)) { ok = false; break; }
+        if (j == nkv - 1) tc5::commit(smem_u32(&o_full[0]));
+      }
+      if (ok && two && issue_pv(1, 2 * nkv - 1, nkv - 1 > 0, nkv - 1)) tc5::commit(smem_u32(&o_full[1]));
       // every MMA this thread issued has completed before TMEM is released
       tc5::commit(smem_u32(drain));
       mbar_drain(drain, 0, 20000000ull);
@@ -347,22 +434,48 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, kErrPrefillWait));
         if (!ok) break;
         tc5::fence_after();
-        float s[kPfBN];
-#pragma unroll
-        for (int c = 0; c < kPfBN / 32; ++c) {
-          float (&chunk)[32] = *reinterpret_cast<float(*)[32]>(&s[c * 32]);
-          tc5::ld32(s_addr + c * 32, chunk);
-        }
-        tc5::wait_ld();
+#if SKV_PF_ONEPASS
         const int n_valid = len_k - j * kPfBN;
+        float sfull[kPfBN];
+#pragma unroll
+        for (int c = 0; c < kPfBN / 32; ++c) tc5::ld32(s_addr + c * 32, *reinterpret_cast<float(*)[32]>(&sfull[c * 32]));
+        tc5::wait_ld();
         if (n_valid < kPfBN) {
 #pragma unroll
           for (int c = 0; c < kPfBN; ++c)
-            if (c >= n_valid) s[c] = -INFINITY;
+            if (c >= n_valid) sfull[c] = -INFINITY;
         }
-        float mx = s[0];
+        float mx8[8];
 #pragma unroll
-        for (int c = 1; c < kPfBN; ++c) mx = fmaxf(mx, s[c]);
+        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(sfull[e], sfull[e + 8]);
+#pragma unroll
+        for (int c = 16; c < kPfBN; c += 16)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], sfull[c + e], sfull[c + 8 + e]);
+#else
+        // pass 1 over S (two halves of 64 columns read from TMEM): the row max
+        const int n_valid = len_k - j * kPfBN;
+        float mx8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+          float sh[64];
+          tc5::ld32(s_addr + hf * 64, *reinterpret_cast<float(*)[32]>(&sh[0]));
+          tc5::ld32(s_addr + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
+          tc5::wait_ld();
+          if (n_valid < kPfBN) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (hf * 64 + c >= n_valid) sh[c] = -INFINITY;
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 16)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], sh[c + e], sh[c + 8 + e]);
+        }
+#endif
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float t_max = fmaf(mx, a.scale_log2, -bias_shift);
         const float m_new = fmaxf(m_run, t_max);
         const bool rescale = m_new > m_run + kPfRescaleThreshold;
@@ -372,37 +485,63 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           m_run = m_new;
         }
         l_run *= alpha;
-        const float neg_bias = -(m_run + bias_shift);
-        float psum = 0.f;
-#pragma unroll
-        for (int c = 0; c < kPfBN / 32; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * e], a.scale_log2, neg_bias));
-            const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * e + 1], a.scale_log2, neg_bias));
-            psum += p0 + p1;
-            pk[e] = pack2<T>(p0, p1);
-          }
-          tc5::st16(s_addr + c * 16, pk);
-        }
-        l_run += psum;
-        tc5::wait_st();
         if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-          // O_t holds the PV products of tiles < j (complete: S_t(j) was issued after them)
+          // correction before this tile's P is published: O_t holds the PV
+          // products of tiles < j, complete since S_t(j) was issued after them
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             float o[32];
             tc5::ld32(o_addr + c * 32, o);
             tc5::wait_ld();
+            const uint64_t al2 = f2_pack(alpha, alpha);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            for (int e = 0; e < 32; e += 2) {
+              const float2 r = f2_unpack(fmul2(f2_pack(o[e], o[e + 1]), al2));
+              o[e] = r.x;
+              o[e + 1] = r.y;
+            }
             tc5::st32(o_addr + c * 32, o);
           }
           tc5::wait_st();
         }
-        tc5::fence_before();
-        mbar_arrive(&p_full[t]);
+        // p = 2^(s * scale*log2(e) - max): P of keys [64h, 64h+64) is packed into
+        // columns [32h, 32h+32) (logits this thread has already read) and
+        // published on its own barrier, so PV can start on the first half
+        const float neg_bias = -(m_run + bias_shift);
+        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
+        const uint64_t nb2 = f2_pack(neg_bias, neg_bias);
+        uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        const bool full_tile = n_valid >= kPfBN;  // masked tails stay on the MUFU (exact zeros)
+#if SKV_PF_ONEPASS
+#pragma unroll
+#else
+#pragma unroll 1
+#endif
+        for (int hf = 0; hf < 2; ++hf) {
+#if SKV_PF_ONEPASS
+          const float (&sh)[64] = *reinterpret_cast<const float(*)[64]>(&sfull[hf * 64]);
+#else
+          float sh[64];
+          tc5::ld32(s_addr + hf * 64, *reinterpret_cast<float(*)[32]>(&sh[0]));
+          tc5::ld32(s_addr + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
+          tc5::wait_ld();
+          if (!full_tile) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (hf * 64 + c >= n_valid) sh[c] = -INFINITY;
+          }
+#endif
+          uint32_t pk[32];
+          if (full_tile) exp_pack_64<true, T>(sh, sc2, nb2, pk, ps2);
+          else exp_pack_64<false, T>(sh, sc2, nb2, pk, ps2);
+          tc5::st16(s_addr + hf * 32, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+          tc5::st16(s_addr + hf * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+          tc5::wait_st();
+          tc5::fence_before();
+          mbar_arrive(&p_half[2 * t + hf]);
+        }
+        const float2 psa = f2_unpack(ps2[0]), psb = f2_unpack(ps2[1]);
+        l_run += (psa.x + psa.y) + (psb.x + psb.y);
       }
 
       // ---------------- epilogue: O / l and LSE for this thread's row

@@ -90,9 +90,9 @@ skv_status skv_device_error(int* code) {
 
 // ------------------------------------------------------------------ planning
 
-skv_status attn_splitkv_plan(int B, int Hq, int Hkv, int Lq, int n, int num_sms, int requested_splits,
+skv_status attn_splitkv_plan(int B, int Hq, int Hkv, int Lq, int n, int D, int num_sms, int requested_splits,
                              int* num_splits, int32_t* bounds) {
-  if (num_splits == nullptr || B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || n < 0 || Hq % Hkv != 0)
+  if (num_splits == nullptr || B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || n < 0 || D < 1 || Hq % Hkv != 0)
     return SKV_ERR_INVALID_ARG;
   if (requested_splits < 0 || requested_splits > skv::kSplitMax) return SKV_ERR_INVALID_ARG;
   int s;
@@ -103,7 +103,7 @@ skv_status attn_splitkv_plan(int B, int Hq, int Hkv, int Lq, int n, int num_sms,
     const int64_t G = Hq / Hkv;
     const int64_t row_groups = skv::ceil_div64(G * Lq, skv::kDecodeRowsPerCta);
     const int64_t units = static_cast<int64_t>(B) * Hkv * row_groups;
-    const int64_t target = static_cast<int64_t>(skv::kCtasPerSm) * num_sms;
+    const int64_t target = static_cast<int64_t>(D > 128 ? skv::kCtasPerSmD256 : skv::kCtasPerSm) * num_sms;
     int64_t ss = std::max<int64_t>(1, skv::ceil_div64(target, units));
     ss = std::min<int64_t>(ss, std::max<int64_t>(1, skv::ceil_div64(n, skv::kSplitMinKeys)));
     ss = std::min<int64_t>(ss, skv::kSplitMax);
@@ -263,7 +263,7 @@ skv_status attn_splitkv_decode(const void* q, const void* k, const void* v, void
   if (splits == 0) {
     const int sms = skv::sm_count();
     if (sms <= 0) return cuda_status(cudaErrorNoDevice);
-    skv_status s = attn_splitkv_plan(B, Hq, Hkv, Lq, Lkv, sms, 0, &splits, nullptr);
+    skv_status s = attn_splitkv_plan(B, Hq, Hkv, Lq, Lkv, D, sms, 0, &splits, nullptr);
     if (s != SKV_OK) return s;
   }
   const size_t need = decode_workspace(B, Hq, Lq, D, splits);
@@ -283,7 +283,7 @@ skv_status attn_splitkv_decode(const void* q, const void* k, const void* v, void
   if (splits > 1) {
     const int64_t rows = static_cast<int64_t>(B) * Hq * Lq;
     e = skv::launch_merge_state(part_o, part_lse, out, lse, splits, 1, 1, static_cast<int>(rows), D, 0, SKV_FP32,
-                                dtype, rows * D, rows, stream);
+                                dtype, rows * D, rows, stream, /*dependent=*/true);
     if (e) return cuda_status(e);
   }
   return SKV_OK;

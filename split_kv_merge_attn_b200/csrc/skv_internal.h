@@ -22,7 +22,8 @@ enum DeviceError : int {
 constexpr int kSplitAlign = 64;
 constexpr int kSplitMinKeys = 128;
 constexpr int kSplitMax = 256;
-constexpr int kCtasPerSm = 2;
+constexpr int kCtasPerSm = 2;       // decode CTAs resident per SM, D <= 128
+constexpr int kCtasPerSmD256 = 1;   // and for D = 256
 constexpr int kDecodeRowsPerCta = 16;
 constexpr int kPrefillRowsPerCta = 256;
 
@@ -34,7 +35,8 @@ int sm_count();  // SM count of the current device (cached per device)
 
 int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, float* lse, int P, int B,
                        int H, int S, int D, int layout_bsh, skv_dtype parts_dt, skv_dtype out_dt,
-                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream);
+                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream,
+                       bool dependent = false);
 
 int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, float* part_o,
                   float* part_lse, const int32_t* kv_len, int B, int Hq, int Hkv, int Lq, int Lkv, int D,

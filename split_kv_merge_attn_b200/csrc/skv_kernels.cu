@@ -106,9 +106,29 @@ int sm_count() {
 
 // ------------------------------------------------------------ merge_state
 
+namespace {
+// Launches the per-row merge as a programmatic dependent of the preceding
+// kernel on the stream when `dependent`: its CTAs may become resident during
+// that kernel's tail and start at its completion (griddepcontrol.wait).
+template <typename TI, typename TO>
+cudaError_t launch_parts(const MergeArgs& a, unsigned rows, cudaStream_t st, bool dependent) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, merge_state_parts_kernel<TI, TO>, a);
+}
+}  // namespace
+
 int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, float* lse, int P, int B, int H,
                        int S, int D, int layout_bsh, skv_dtype parts_dt, skv_dtype out_dt,
-                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream) {
+                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream, bool dependent) {
   MergeArgs a;
   a.o_parts = o_parts;
   a.lse_parts = lse_parts;
@@ -131,7 +151,14 @@ int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, f
   const int64_t cap = static_cast<int64_t>(sms > 0 ? sms : 148) * 8;  // 8 x 256 threads per SM resident
   if (blocks > cap) blocks = cap;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-#define SKV_MERGE(TI, TO) merge_state_kernel<TI, TO><<<static_cast<unsigned>(blocks), threads, 0, st>>>(a)
+  // few rows and many parts: one CTA per row, parallel over the parts
+  const bool per_row = P >= 8 && rows <= 4096 && D <= 2048;
+  cudaError_t le = cudaSuccess;
+#define SKV_MERGE(TI, TO)                                                                   \
+  do {                                                                                      \
+    if (per_row) le = launch_parts<TI, TO>(a, static_cast<unsigned>(rows), st, dependent); \
+    else merge_state_kernel<TI, TO><<<static_cast<unsigned>(blocks), threads, 0, st>>>(a); \
+  } while (0)
   if (parts_dt == SKV_FP32 && out_dt == SKV_BF16) SKV_MERGE(float, __nv_bfloat16);
   else if (parts_dt == SKV_FP32 && out_dt == SKV_FP16) SKV_MERGE(float, __half);
   else if (parts_dt == SKV_FP32 && out_dt == SKV_FP32) SKV_MERGE(float, float);
@@ -143,6 +170,7 @@ int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, f
   else if (parts_dt == SKV_FP16 && out_dt == SKV_BF16) SKV_MERGE(__half, __nv_bfloat16);
   else return cudaErrorInvalidValue;
 #undef SKV_MERGE
+  if (le != cudaSuccess) return le;
   return counted(cudaGetLastError(), 1);
 }
 

@@ -154,11 +154,12 @@ def test_split_plan_matches_oracle_bit_exact():
         cases.append((int(rng.integers(1, 9)), hkv * int(rng.integers(1, 9)), hkv, int(rng.integers(1, 9)),
                       int(rng.integers(0, 70000)), int(rng.integers(1, 200))))
     for (B, Hq, Hkv, Lq, n, sms) in cases:
-        s, bounds = skv.attn_splitkv_plan(B, Hq, Hkv, Lq, n, sms, 0)
-        assert s == O.auto_num_splits(B, Hkv, Hq, Lq, n, sms), (B, Hq, Hkv, Lq, n, sms)
-        assert bounds == O.split_bounds(n, s)
+        for D in (64, 128, 256):
+            s, bounds = skv.attn_splitkv_plan(B, Hq, Hkv, Lq, n, D, sms, 0)
+            assert s == O.auto_num_splits(B, Hkv, Hq, Lq, n, sms, D=D), (B, Hq, Hkv, Lq, n, sms, D)
+            assert bounds == O.split_bounds(n, s)
         for req in (1, 3, 37, 256):
-            s2, b2 = skv.attn_splitkv_plan(B, Hq, Hkv, Lq, n, sms, req)
+            s2, b2 = skv.attn_splitkv_plan(B, Hq, Hkv, Lq, n, 128, sms, req)
             assert s2 == req and b2 == O.split_bounds(n, req)
 
 

@@ -22,7 +22,7 @@ def run_decode(d, num_splits=0, kv_len=None, poison=True):
     splits = num_splits
     if splits == 0:
         sms = torch.cuda.get_device_properties(0).multi_processor_count
-        splits, _ = skv.attn_splitkv_plan(B, Hq, k.shape[1], Lq, k.shape[2], sms, 0)
+        splits, _ = skv.attn_splitkv_plan(B, Hq, k.shape[1], Lq, k.shape[2], D, sms, 0)
     ws = skv.attn_splitkv_workspace(B, Hq, Lq, D, splits)
     workspace = torch.full((max(ws, 1),), 0xFF, dtype=torch.uint8, device="cuda")  # NaN bit patterns
     kl = None if kv_len is None else torch.tensor(kv_len, dtype=torch.int32, device="cuda")

@@ -426,10 +426,14 @@ def test_split_plan_hand_values():
     assert O.split_bounds(32768, 37)[-2] == 36 * 896
     # Lkv = 4096: 37 capped to ceil(4096/128) = 32; C = 128 -> 32 splits
     assert O.auto_num_splits(1, 8, 32, 1, 4096, 148) == 32
-    # D256 shape (4 kv heads, G*Lq = 16): ceil(296/4) = 74, Lkv 16384 -> C = 256 -> 64
+    # D=128 rule on a 4-kv-head shape (G*Lq = 16): ceil(296/4) = 74, Lkv 16384 -> C = 256 -> 64
     assert O.auto_num_splits(1, 4, 16, 4, 16384, 148) == 64
     # G*Lq = 32 rows -> two row groups per kv head
     assert O.auto_num_splits(1, 4, 16, 8, 16384, 148) == 37
+    # D = 256 aims at one CTA per SM: ceil(148/4) = 37, C = roundup(443, 64) = 448 -> 37
+    assert O.auto_num_splits(1, 4, 16, 4, 16384, 148, D=256) == 37
+    # two row groups: ceil(148/8) = 19, C = roundup(863, 64) = 896 -> ceil(16384/896) = 19
+    assert O.auto_num_splits(1, 4, 16, 8, 16384, 148, D=256) == 19
     assert O.auto_num_splits(1, 8, 32, 1, 0, 148) == 1
     assert O.auto_num_splits(1, 8, 32, 1, 100, 148) == 1
 
