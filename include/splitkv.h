@@ -178,6 +178,31 @@ skv_status attn_splitkv_plan(int B, int Hq, int Hkv, int Lq, int n, int D, int n
 /* Workspace bytes for a decode with this many splits (fp32 partial O and LSE). */
 size_t attn_splitkv_workspace(int B, int Hq, int Lq, int D, int num_splits);
 
+/* attn_splitkv_decode_static: the same decode for callers that cannot
+ * allocate device memory (code running under an allocator that owns all device
+ * memory, plugins handed only their input and output buffers, hosts that
+ * forbid allocation after start-up).  The source pages describe no such entry
+ * point; it exists for those callers.
+ *
+ * Arguments and results are those of attn_splitkv_decode without the
+ * workspace: the per-split partials go to a fixed 8 MiB array in device global
+ * memory that the library defines (every GPU that loads the library holds it
+ * until the process exits).  Nothing is allocated: no cudaMalloc, cudaFree or
+ * allocating library call.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - A problem whose partials need more than 8 MiB
+ *     (attn_splitkv_workspace(B, Hq, Lq, D, splits) > 8 MiB) is refused with
+ *     SKV_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *   - Every call shares the one array and it keeps the last call's contents;
+ *     nothing in it needs to start at zero (each call writes every partial
+ *     slot it reads).  Calls that overlap on the GPU (other streams, other host
+ *     threads) race on it and must be serialised by the caller. */
+skv_status attn_splitkv_decode_static(const void* q, const void* k, const void* v, void* out,
+                                      float* lse, int B, int Hq, int Hkv, int Lq, int Lkv, int D,
+                                      float scale, skv_dtype dtype, const int32_t* kv_len,
+                                      int num_splits, skv_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* merge_state: combine P partial (O, LSE) results of disjoint KV ranges.    */
 /*

@@ -37,6 +37,8 @@ SIGNATURES = {
     "attn_varlen_plan": (_c_int, [_vp, _vp, _c_int, _c_int, _vp, _vp]),
     "attn_splitkv_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_float, _c_int, _vp, _c_int, _vp, _c_size, _vp]),
+    "attn_splitkv_decode_static": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                            _c_float, _c_int, _vp, _c_int, _vp]),
     "attn_splitkv_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "attn_splitkv_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "merge_state": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -260,6 +262,30 @@ def attn_splitkv_decode(q, k, v, scale: Optional[float] = None, kv_len=None, num
     return out, lse
 
 
+def attn_splitkv_decode_static(q, k, v, scale: Optional[float] = None, kv_len=None, num_splits: int = 0,
+                               out=None, lse=None, return_lse: bool = True, stream=None):
+    """attn_splitkv_decode for callers that cannot allocate device memory: the
+    per-split partials live in the library's fixed 8 MiB device array (no
+    workspace).  This wrapper allocates out/lse only if they are not given."""
+    torch = _torch()
+    _need_cuda(q, k, v, out, lse, kv_len)
+    B, Hq, Lq, D = q.shape
+    _, Hkv, Lkv, _ = k.shape
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    if not return_lse:
+        lse = None
+    st = lib().attn_splitkv_decode_static(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lkv, D,
+                                          float(scale), _dtype_code(q), _ptr(kv_len), int(num_splits),
+                                          _stream(stream, q.device))
+    _check(st, "attn_splitkv_decode_static")
+    return out, lse
+
+
 def merge_state(o_parts, lse_parts, layout: str = "HND", out=None, lse=None, out_dtype=None,
                 return_lse: bool = True, stream=None):
     """Merge P partial results.  o_parts [P,B,H,S,D] (HND), [P,B,S,H,D] (NHD)
@@ -288,6 +314,6 @@ def merge_state(o_parts, lse_parts, layout: str = "HND", out=None, lse=None, out
     return out, lse
 
 
-__all__ = ["attn_fwd_lse", "attn_splitkv_decode", "merge_state", "attn_splitkv_plan", "attn_splitkv_workspace",
+__all__ = ["attn_fwd_lse", "attn_splitkv_decode", "attn_splitkv_decode_static", "merge_state", "attn_splitkv_plan", "attn_splitkv_workspace",
            "attn_fwd_lse_workspace", "attn_varlen_plan", "device_error", "launch_count", "lib", "SkvError", "status_string",
            "LIB_PATH", "SIGNATURES"]
