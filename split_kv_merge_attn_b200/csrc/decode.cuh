@@ -102,23 +102,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // ---- Q rows of this group into shared memory (zero rows pad the tile)
-  {
-    constexpr int vpr = D / 8;
-    for (int v = tid; v < kDecodeRows * vpr; v += kDecodeThreads) {
-      const int r = v / vpr, c = v % vpr;
-      const int rglob = rg * kDecodeRows + r;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (rglob < rows_total) {
-        const int h = hkv * G + rglob / a.Lq;
-        const int i = rglob % a.Lq;
-        const T* src = static_cast<const T*>(a.q) + ((static_cast<int64_t>(b) * a.Hq + h) * a.Lq + i) * D + c * 8;
-        val = *reinterpret_cast<const uint4*>(src);
-      }
-      *reinterpret_cast<uint4*>(qs + r * Cfg::kQStride + c * 8) = val;
-    }
-  }
-  __syncthreads();
+  __syncthreads();  // barriers initialised
   // let a programmatically dependent merge launch be scheduled; it still waits
   // for this whole grid to finish before it reads the partials
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -157,6 +141,24 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
   }
 
   // ================= consumer warps
+  // Q rows of this group into shared memory (zero rows pad the tile); the
+  // producer's first K/V loads are already in flight meanwhile
+  {
+    constexpr int vpr = D / 8;
+    for (int v = tid; v < kDecodeRows * vpr; v += kDecodeConsumerWarps * 32) {
+      const int r = v / vpr, c = v % vpr;
+      const int rglob = rg * kDecodeRows + r;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (rglob < rows_total) {
+        const int h = hkv * G + rglob / a.Lq;
+        const int i = rglob % a.Lq;
+        const T* src = static_cast<const T*>(a.q) + ((static_cast<int64_t>(b) * a.Hq + h) * a.Lq + i) * D + c * 8;
+        val = *reinterpret_cast<const uint4*>(src);
+      }
+      *reinterpret_cast<uint4*>(qs + r * Cfg::kQStride + c * 8) = val;
+    }
+  }
+  named_barrier_sync(1, kDecodeConsumerWarps * 32);
   const int g = lane >> 2, tq = lane & 3;
   const uint32_t qs_addr = smem_u32(qs);
   uint32_t qa[Cfg::kQInRegs ? D / 16 : 1][4];

@@ -7,9 +7,7 @@
 // cross-split reduce of the ExecuTorch split-K PR.  That PR's review measured a
 // reduce parallel over rows only, with two exponentials on the loop-carried
 // chain, as latency bound; here every thread owns one 16-byte slice of one
-// row (parallel over rows x D), the max is a separate first pass over the P
-// LSE values, and the weights are independent, so no exponential sits on a
-// serial dependency chain.
+// row (parallel over rows x D) and requests all of its parts at once.
 #pragma once
 
 #include "skv_device.cuh"
@@ -57,6 +55,38 @@ struct Vec8<__nv_bfloat16> : Vec8Half<__nv_bfloat16> {};
 template <>
 struct Vec8<__half> : Vec8Half<__half> {};
 
+// Eight elements kept as the raw 16-byte words they were loaded as (one word
+// for 16-bit types, two for fp32) until they are used: fewer live registers
+// than unpacked floats, so more loads can be in flight per SM.
+template <typename T>
+struct Raw8 {
+  static constexpr int kWords = sizeof(T) == 4 ? 2 : 1;
+  uint4 w[kWords];
+  __device__ __forceinline__ void load(const T* p) {
+#pragma unroll
+    for (int i = 0; i < kWords; ++i) w[i] = __ldg(reinterpret_cast<const uint4*>(p) + i);
+  }
+  __device__ __forceinline__ void unpack(float (&x)[8]) const {
+    if constexpr (sizeof(T) == 4) {
+      const float* f0 = reinterpret_cast<const float*>(&w[0]);
+      const float* f1 = reinterpret_cast<const float*>(&w[1]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[e] = f0[e];
+        x[4 + e] = f1[e];
+      }
+    } else {
+      const uint32_t u[4] = {w[0].x, w[0].y, w[0].z, w[0].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = unpack2<T>(u[e]);
+        x[2 * e] = f.x;
+        x[2 * e + 1] = f.y;
+      }
+    }
+  }
+};
+
 struct MergeArgs {
   const void* o_parts;
   const float* lse_parts;
@@ -71,67 +101,57 @@ struct MergeArgs {
 
 template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) merge_state_kernel(MergeArgs a) {
+  // one thread per 8-element slice of one row; the loads of up to kBatch parts
+  // (LSE and O slice) are issued together and merged with a running max, so a
+  // thread waits for memory once per kBatch parts, not once per part
+  constexpr int kBatch = 4;
   const TI* __restrict__ op = static_cast<const TI*>(a.o_parts);
   const float* __restrict__ lp = a.lse_parts;
   TO* __restrict__ out = static_cast<TO*>(a.out);
   const int vpr = a.D >> 3;  // 8-element vectors per row
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < a.n_vec; g += stride) {
-    const int64_t row = g / vpr;          // row in O's memory order
-    const int c = static_cast<int>(g - row * vpr);
-    int64_t lrow = row;                   // row in the [B, H, S] LSE order
-    if (a.layout_bsh) {
-      const int h = static_cast<int>(row % a.H);
-      const int64_t bs = row / a.H;
-      const int s = static_cast<int>(bs % a.S);
-      const int64_t b = bs / a.S;
-      lrow = (b * a.H + h) * a.S + s;
-    }
-    // pass 1: the max over parts (independent loads)
-    float M = -INFINITY;
-    for (int p = 0; p < a.P; ++p) M = fmaxf(M, __ldg(lp + p * a.part_stride_lse + lrow));
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    float W = 0.f;
-    if (M != -INFINITY) {
-      // pass 2: weights and the weighted sum; parts of weight 0 are skipped
-      const TI* base = op + row * a.D + c * 8;
-      int p = 0;
-      for (; p + 2 <= a.P; p += 2) {
-        const float w0 = exp2f(__ldg(lp + p * a.part_stride_lse + lrow) - M);
-        const float w1 = exp2f(__ldg(lp + (p + 1) * a.part_stride_lse + lrow) - M);
-        float x0[8], x1[8];
-        if (w0 > 0.f) Vec8<TI>::load(base + p * a.part_stride_o, x0);
-        if (w1 > 0.f) Vec8<TI>::load(base + (p + 1) * a.part_stride_o, x1);
-        if (w0 > 0.f) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] = fmaf(w0, x0[e], acc[e]);
-          W += w0;
-        }
-        if (w1 > 0.f) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] = fmaf(w1, x1[e], acc[e]);
-          W += w1;
-        }
-      }
-      for (; p < a.P; ++p) {
-        const float w = exp2f(__ldg(lp + p * a.part_stride_lse + lrow) - M);
-        if (w > 0.f) {
-          float x[8];
-          Vec8<TI>::load(base + p * a.part_stride_o, x);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, x[e], acc[e]);
-          W += w;
-        }
-      }
-      const float inv = 1.0f / W;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] *= inv;
-    }
-    Vec8<TO>::store(out + row * a.D + c * 8, acc);
-    if (c == 0 && a.lse != nullptr) a.lse[lrow] = (M == -INFINITY) ? -INFINITY : M + log2f(W);
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (g >= a.n_vec) return;
+  const int64_t row = g / vpr;          // row in O's memory order
+  const int c = static_cast<int>(g - row * vpr);
+  int64_t lrow = row;                   // row in the [B, H, S] LSE order
+  if (a.layout_bsh) {
+    const int h = static_cast<int>(row % a.H);
+    const int64_t bs = row / a.H;
+    const int s = static_cast<int>(bs % a.S);
+    const int64_t b = bs / a.S;
+    lrow = (b * a.H + h) * a.S + s;
   }
+  const TI* base = op + row * a.D + c * 8;
+  float m = -INFINITY, W = 0.f;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int p0 = 0; p0 < a.P; p0 += kBatch) {
+    float L[kBatch];
+    Raw8<TI> x[kBatch];
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      const int p = p0 + r;
+      L[r] = (p < a.P) ? __ldg(lp + p * a.part_stride_lse + lrow) : -INFINITY;
+      if (p < a.P) x[r].load(base + p * a.part_stride_o);
+    }
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      if (L[r] == -INFINITY) continue;   // an empty part carries no weight; its O slot is not used
+      const float mn = fmaxf(m, L[r]);
+      const float sc = exp2f(m - mn);    // 0 while m is -inf
+      const float w = exp2f(L[r] - mn);
+      float xf[8];
+      x[r].unpack(xf);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, xf[e], acc[e] * sc);
+      W = W * sc + w;
+      m = mn;
+    }
+  }
+  const float inv = (m != -INFINITY && W > 0.f) ? 1.0f / W : 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] *= inv;
+  Vec8<TO>::store(out + row * a.D + c * 8, acc);
+  if (c == 0 && a.lse != nullptr) a.lse[lrow] = (m == -INFINITY) ? -INFINITY : m + log2f(W);
 }
 
 // Variant for few rows and many parts (the cross-split reduce of a decode:

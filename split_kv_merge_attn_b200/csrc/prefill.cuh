@@ -116,7 +116,8 @@ struct PrefillCfg {
   // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_half[2][2], o_full[2], drain
   static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + TMEM slot, abort flag; + alignment pad
+  static constexpr int kOffMu = kOffMisc + 16;             // [2][D] fp32 mean of K (smooth_k)
+  static constexpr int kSmemBytes = kOffMu + 2 * D * 4 + 1024;  // + alignment pad
   static constexpr int kSCol0 = 0, kSCol1 = 128, kOCol0 = 256, kOCol1 = 256 + D;
   static constexpr uint32_t kTmemCols = 512;
 };
@@ -124,7 +125,8 @@ struct PrefillCfg {
 struct PrefillArgs {
   void* out;
   float* lse;
-  const float* kmean;   // smooth: [Bseq, Hkv, D] fp32, else null
+  const float* kmean;   // smooth (materialised K'): [Bseq, Hkv, D] fp32 mean, else null
+  const float* kpartial;  // smooth (logit shift): [chunks, Bseq, Hkv, D] per-256-key column sums, else null
   int shift_logits;     // smooth: 1 = subtract the mean term from the fp32 logits (K unsmoothed),
                         //         0 = K was replaced by K' = K - mean (already smoothed)
   const int* cu_q;
@@ -400,10 +402,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
       // smooth_k: delta = scale*log2(e) * (q_i . mean(K)), the shift smoothing removes
       float delta = 0.f;
-      if (a.kmean != nullptr) {
+      if (a.kmean != nullptr || a.kpartial != nullptr) {
+        const float* mu;
+        if (a.kpartial != nullptr) {
+          // mean over this call's KV range from the per-256-key column sums
+          float* mu_s = reinterpret_cast<float*>(smem + Cfg::kOffMu) + t * D;
+          if (row < D) {
+            const int nch = (len_k + 255) / 256;
+            float sum = 0.f;
+            for (int c = 0; c < nch; ++c)
+              sum += __ldg(a.kpartial + ((static_cast<int64_t>(c) * a.B + b) * a.Hkv + hkv) * D + row);
+            mu_s[row] = sum / static_cast<float>(len_k);
+          }
+          named_barrier_sync(1 + t, kPfBM);
+          mu = mu_s;
+        } else {
+          mu = a.kmean + (static_cast<int64_t>(b) * a.Hkv + hkv) * D;
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, kErrPrefillWait));
         if (ok) {
-          const float* mu = a.kmean + (static_cast<int64_t>(b) * a.Hkv + hkv) * D;
           float acc = 0.f;
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
@@ -416,8 +433,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               for (int e = 0; e < 4; ++e) {
                 const float2 f = unpack2<T>(w[e]);
                 const int d = bx * 64 + c * 8 + 2 * e;
-                acc = fmaf(f.x, __ldg(mu + d), acc);
-                acc = fmaf(f.y, __ldg(mu + d + 1), acc);
+                acc = fmaf(f.x, mu[d], acc);
+                acc = fmaf(f.y, mu[d + 1], acc);
               }
             }
           }

@@ -232,9 +232,13 @@ skv_status attn_fwd_lse(const void* q, const void* k, const void* v, void* out, 
     int e = skv::launch_smooth_k(k, kprime, kmean, partial, varlen ? cu_seqlens_k : nullptr, B, Hkv, Sk, max_len,
                                  D, dtype, layout, stream);
     if (e) return cuda_status(e);
-    p.kmean = kmean;
+    if (smooth_k == 1) {
+      p.kpartial = partial;   // the prefill kernel sums these into the mean itself
+    } else {
+      p.kmean = kmean;
+      p.k = kprime;
+    }
     p.shift_logits = smooth_k == 1 ? 1 : 0;
-    if (smooth_k == 2) p.k = kprime;
   }
   return cuda_status(skv::launch_prefill(p, stream));
 }

@@ -48,7 +48,8 @@ struct PrefillLaunch {
   const void* v;
   void* out;
   float* lse;
-  const float* kmean;      // [B(or seqs), Hkv, D] fp32 when smooth_k, else null
+  const float* kmean;      // [B(or seqs), Hkv, D] fp32 mean (materialised smooth_k), else null
+  const float* kpartial;   // [chunks, B(or seqs), Hkv, D] per-256-key sums (shift smooth_k), else null
   int shift_logits;        // smooth_k == 1: apply the mean shift to the logits
   const int32_t* cu_q;     // device, varlen only
   const int32_t* cu_k;
@@ -65,9 +66,9 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream);
 int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int32_t* order,
                        int32_t* offsets, skv_stream_t stream);
 
-// smooth_k prepass: fp32 mean over each (batch or sequence, kv head) KV range
-// into kmean [B, Hkv, D] (via per-256-key partial sums in `partial`), and, if
-// k_smoothed != null, K' = K - mean rounded to the input type.
+// smooth_k prepass: fp32 per-256-key column sums of K for each (batch or
+// sequence, kv head) into `partial`; if k_smoothed != null also the mean
+// kmean [B, Hkv, D] and K' = K - mean rounded to the input type.
 int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partial, const int32_t* cu_k, int B,
                     int Hkv, int Sk, int max_len, int D, skv_dtype dt, skv_layout layout, skv_stream_t stream);
 

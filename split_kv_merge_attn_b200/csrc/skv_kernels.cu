@@ -147,12 +147,11 @@ int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, f
   if (a.n_vec == 0) return 0;
   const int threads = 256;
   const int sms = sm_count();
-  int64_t blocks = (a.n_vec + threads - 1) / threads;
-  const int64_t cap = static_cast<int64_t>(sms > 0 ? sms : 148) * 8;  // 8 x 256 threads per SM resident
-  if (blocks > cap) blocks = cap;
+  const int64_t blocks = (a.n_vec + threads - 1) / threads;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // few rows and many parts: one CTA per row, parallel over the parts
-  const bool per_row = P >= 8 && rows <= 4096 && D <= 2048;
+  const bool per_row = P >= 8 && rows <= 4096 && D <= 2048 && sms > 0;
   cudaError_t le = cudaSuccess;
 #define SKV_MERGE(TI, TO)                                                                   \
   do {                                                                                      \
@@ -286,6 +285,7 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   a.out = p.out;
   a.lse = p.lse;
   a.kmean = p.kmean;
+  a.kpartial = p.kpartial;
   a.shift_logits = p.shift_logits;
   a.cu_q = p.cu_q;
   a.cu_k = p.cu_k;
@@ -322,7 +322,10 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
 
 int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int32_t* order, int32_t* offsets,
                        skv_stream_t stream) {
-  varlen_plan_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(cu_q, cu_k, B, Hq, order, offsets);
+  // one block; no more threads than sequences (rounded to a warp): the final
+  // scan walks one partial sum per thread
+  const int threads = B >= 1024 ? 1024 : ((B + 31) / 32) * 32;
+  varlen_plan_kernel<<<1, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(cu_q, cu_k, B, Hq, order, offsets);
   return counted(cudaGetLastError(), 1);
 }
 
@@ -348,13 +351,16 @@ int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partia
     if (dt == SKV_BF16) kmean_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
     else kmean_partial_kernel<__half><<<grid, 256, 0, st>>>(a);
   }
-  kmean_finalize_kernel<<<B * Hkv, D, 0, st>>>(a);
+  // the mean itself is needed here only to materialise K'; otherwise the
+  // prefill kernel adds up the per-chunk partial sums of its own KV range
+  if (k_smoothed != nullptr) kmean_finalize_kernel<<<B * Hkv, D, 0, st>>>(a);
   if (k_smoothed != nullptr && a.nchunks > 0) {
     dim3 grid(a.nchunks, B, Hkv);
     if (dt == SKV_BF16) ksmooth_write_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
     else ksmooth_write_kernel<__half><<<grid, 256, 0, st>>>(a);
   }
-  const int n = 1 + (a.nchunks > 0 ? 1 : 0) + (k_smoothed != nullptr && a.nchunks > 0 ? 1 : 0);
+  const int n = (a.nchunks > 0 ? 1 : 0) + (k_smoothed != nullptr ? 1 : 0) +
+                (k_smoothed != nullptr && a.nchunks > 0 ? 1 : 0);
   return counted(cudaGetLastError(), n);
 }
 

@@ -37,7 +37,8 @@ __device__ __forceinline__ int smooth_len(const SmoothArgs& a, int b) {
   return a.layout == 2 ? a.cu_k[b + 1] - a.cu_k[b] : a.Sk;
 }
 
-// grid (nchunks, Bseq, Hkv), 256 threads: (D/8) column vectors x (256/(D/8)) row lanes
+// grid (nchunks, Bseq, Hkv), 256 threads: (D/8) column vectors x (256/(D/8)) row lanes.
+// Every thread issues its row loads in batches of 8 before summing them.
 template <typename T>
 __global__ void __launch_bounds__(256) kmean_partial_kernel(SmoothArgs a) {
   const int c = blockIdx.x, b = blockIdx.y, hkv = blockIdx.z;
@@ -48,14 +49,24 @@ __global__ void __launch_bounds__(256) kmean_partial_kernel(SmoothArgs a) {
   const int s0 = c * kSmoothChunk, s1 = min(len, s0 + kSmoothChunk);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   const T* k = static_cast<const T*>(a.k);
-  for (int s = s0 + rl; s < s1; s += lanes) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(k + smooth_row_off(a, b, hkv, s) + cv * 8));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  // rows of this thread: s0 + rl + i * lanes; loads issued in batches of 8
+  for (int i0 = 0; i0 * lanes < kSmoothChunk; i0 += 8) {
+    uint4 u[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = unpack2<T>(w[e]);
-      acc[2 * e] += f.x;
-      acc[2 * e + 1] += f.y;
+    for (int i = 0; i < 8; ++i) {
+      const int s = s0 + rl + (i0 + i) * lanes;
+      u[i] = (s < s1) ? __ldg(reinterpret_cast<const uint4*>(k + smooth_row_off(a, b, hkv, s) + cv * 8))
+                      : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = unpack2<T>(w[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
     }
   }
   __shared__ float red[256 * 8];
