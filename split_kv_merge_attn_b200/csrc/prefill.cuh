@@ -41,13 +41,10 @@ constexpr int kPfBN = 128;          // keys per KV tile
 constexpr int kPfThreads = 320;
 constexpr float kPfRescaleThreshold = 8.0f;
 
-// Tuning switches (compile time).  SKV_PF_ONEPASS: S is read from TMEM once
-// (128 registers of logits per thread) instead of twice in halves.
-// SKV_PF_POLY_PAIRS: of every 16 pairs of probabilities, this many are
-// computed with the FMA-pipe polynomial below instead of the MUFU ex2.
-#ifndef SKV_PF_ONEPASS
-#define SKV_PF_ONEPASS 0
-#endif
+// Tuning switch (compile time).  SKV_PF_POLY_PAIRS: of every 16 pairs of
+// probabilities, this many are computed with the FMA-pipe polynomial below
+// instead of the MUFU ex2 (0 by default: measured slower on B200, where the
+// softmax is latency- rather than MUFU-bound).
 #ifndef SKV_PF_POLY_PAIRS
 #define SKV_PF_POLY_PAIRS 0
 #endif
@@ -451,25 +448,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, kErrPrefillWait));
         if (!ok) break;
         tc5::fence_after();
-#if SKV_PF_ONEPASS
-        const int n_valid = len_k - j * kPfBN;
-        float sfull[kPfBN];
-#pragma unroll
-        for (int c = 0; c < kPfBN / 32; ++c) tc5::ld32(s_addr + c * 32, *reinterpret_cast<float(*)[32]>(&sfull[c * 32]));
-        tc5::wait_ld();
-        if (n_valid < kPfBN) {
-#pragma unroll
-          for (int c = 0; c < kPfBN; ++c)
-            if (c >= n_valid) sfull[c] = -INFINITY;
-        }
-        float mx8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(sfull[e], sfull[e + 8]);
-#pragma unroll
-        for (int c = 16; c < kPfBN; c += 16)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], sfull[c + e], sfull[c + 8 + e]);
-#else
         // pass 1 over S (two halves of 64 columns read from TMEM): the row max
         const int n_valid = len_k - j * kPfBN;
         float mx8[8];
@@ -491,7 +469,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], sh[c + e], sh[c + 8 + e]);
         }
-#endif
         const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float t_max = fmaf(mx, a.scale_log2, -bias_shift);
         const float m_new = fmaxf(m_run, t_max);
@@ -529,15 +506,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint64_t nb2 = f2_pack(neg_bias, neg_bias);
         uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
         const bool full_tile = n_valid >= kPfBN;  // masked tails stay on the MUFU (exact zeros)
-#if SKV_PF_ONEPASS
-#pragma unroll
-#else
 #pragma unroll 1
-#endif
         for (int hf = 0; hf < 2; ++hf) {
-#if SKV_PF_ONEPASS
-          const float (&sh)[64] = *reinterpret_cast<const float(*)[64]>(&sfull[hf * 64]);
-#else
           float sh[64];
           tc5::ld32(s_addr + hf * 64, *reinterpret_cast<float(*)[32]>(&sh[0]));
           tc5::ld32(s_addr + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
@@ -547,7 +517,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int c = 0; c < 64; ++c)
               if (hf * 64 + c >= n_valid) sh[c] = -INFINITY;
           }
-#endif
           uint32_t pk[32];
           if (full_tile) exp_pack_64<true, T>(sh, sc2, nb2, pk, ps2);
           else exp_pack_64<false, T>(sh, sc2, nb2, pk, ps2);
