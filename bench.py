@@ -131,6 +131,36 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 
+def init_distributed(world: int, backend: str = "nccl", timeout_s: int = 120):
+    """One process per GPU under torchrun: binds LOCAL_RANK's device (nccl)
+    and joins the process group with a short timeout, so ranks that wait for
+    a lost peer end with an error.  Returns torch.distributed, or None at N=1."""
+    if world <= 1:
+        return None
+    import datetime
+    import torch
+    import torch.distributed as tdist
+    if backend == "nccl":
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    tdist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return tdist
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The step time the job reports: the slowest rank's (identity at N=1)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(flops_per_rank_step: float, world: int, ms: float) -> float:
+    """Whole-job TFLOP/s: the units every rank processed / the max-over-ranks time."""
+    return flops_per_rank_step * world / (ms * 1e-3) / 1e12
+
+
 def run_ours(args, rank, world, dist):
     import torch
     import split_kv_merge_attn_b200 as skv
@@ -250,12 +280,8 @@ def run_ours(args, rank, world, dist):
     clocks = sampler.stop() if sampler else None
     step_ms = [evs[i][0].elapsed_time(evs[i][n_ev - 1]) for i in range(args.steps)]
     part_ms = {p: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)] for j, p in enumerate(parts)}
-    ms = sum(step_ms) / len(step_ms)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = step_flops * world / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), dist, dev)
+    value = job_value(step_flops, world, ms)
     assert skv.device_error() == 0
 
     # ---------------- dominant kernel roofline: the varlen prefill launch
@@ -397,12 +423,8 @@ def run_e2e(args, dev, host, skv, torch, step_flops, world, dist):
         e2e_step()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / n
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(step_flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, dist, dev)
+    return {"value": round(job_value(step_flops, world, ms), 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 3),
             "steps": n}
 
@@ -461,7 +483,8 @@ def run_reference(args, rank, world):
     same workload on the host cores."""
     if rank != 0:
         return
-    per_step = max(2.0, min(20.0, 60.0 / max(args.steps + args.warmup, 1)))
+    # each step a bounded sample: the whole run stays near a minute
+    per_step = max(0.2, min(args.cpu_seconds, 60.0 / max(args.steps + args.warmup, 1)))
     for _ in range(args.warmup):
         oracle_sample(per_step)
     fl, secs = 0, 0.0
@@ -544,14 +567,7 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
-    import torch
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as tdist
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        dist = tdist
+    dist = init_distributed(world, "nccl")
     try:
         run_ours(args, rank, world, dist)
     finally:
