@@ -175,8 +175,38 @@ skv_status attn_splitkv_decode(const void* q, const void* k, const void* v, void
 skv_status attn_splitkv_plan(int B, int Hq, int Hkv, int Lq, int n, int D, int num_sms,
                              int requested_splits, int* num_splits, int32_t* bounds);
 
-/* Workspace bytes for a decode with this many splits (fp32 partial O and LSE). */
+/* Workspace bytes for a decode with this many splits: fp32 partial O and LSE
+ * plus the arrival counters attn_splitkv_decode_fused uses (0 for one split). */
 size_t attn_splitkv_workspace(int B, int Hq, int Lq, int D, int num_splits);
+
+/* attn_splitkv_decode_fused: the same decode in ONE kernel launch.
+ *
+ * The single-launch variant of the split-KV decode: the cross-split reduce of
+ * the ExecuTorch split-K PR (and the merge formula of merge_state) runs inside
+ * the decode kernel.  Each CTA writes its split's partial (O, LSE) and then
+ * increments the arrival counter of its (batch, kv head, row group); the CTA
+ * that brings the counter to num_splits merges the group's partials, writes
+ * out and lse, and sets the counter back to zero.  No CTA waits for another.
+ * Results equal attn_splitkv_decode's up to fp32 rounding order.
+ *
+ * Arguments as attn_splitkv_decode.  The workspace's counter region must be
+ * zero before the first call on a workspace: zero the whole workspace once
+ * (attn_splitkv_workspace_init, or any memset).  Every call that completes
+ * without a device error leaves it zero again, so one zeroed workspace serves
+ * any number of calls and CUDA-graph replays on one stream.  After a device
+ * error (skv_device_error), zero it again.  A counter found non-zero on
+ * arrival records device error 0x103.  Calls that overlap on the GPU must use
+ * different workspaces. */
+skv_status attn_splitkv_decode_fused(const void* q, const void* k, const void* v, void* out,
+                                     float* lse, int B, int Hq, int Hkv, int Lq, int Lkv, int D,
+                                     float scale, skv_dtype dtype, const int32_t* kv_len,
+                                     int num_splits, void* workspace, size_t workspace_bytes,
+                                     skv_stream_t stream);
+
+/* Zeroes `workspace_bytes` bytes of a decode workspace on `stream`
+ * (cudaMemsetAsync): the one-time preparation attn_splitkv_decode_fused needs.
+ * NULL with 0 bytes is a no-op. */
+skv_status attn_splitkv_workspace_init(void* workspace, size_t workspace_bytes, skv_stream_t stream);
 
 /* attn_splitkv_decode_static: the same decode for callers that cannot
  * allocate device memory (code running under an allocator that owns all device

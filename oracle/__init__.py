@@ -253,8 +253,8 @@ def lse_varlen_to_dense(lse_ht: np.ndarray, B: int, S: int) -> np.ndarray:
 SPLIT_ALIGN = 64          # split chunk is a multiple of this many keys
 SPLIT_MIN_KEYS = 128      # the automatic plan keeps at least this many keys per split
 SPLIT_MAX = 256           # upper limit on the number of splits
-CTAS_PER_SM = 2           # the automatic plan aims for this many CTAs per SM (D <= 128) ...
-CTAS_PER_SM_D256 = 1      # ... and this many for D = 256 (one decode CTA fills an SM)
+CTAS_PER_SM = (1, 1)      # the automatic plan aims for num/den decode CTAs per SM (D <= 128) ...
+CTAS_PER_SM_D256 = (2, 3) # ... and for D = 256 (whose CTA holds twice the bytes in flight)
 DECODE_ROWS_PER_CTA = 16  # query rows (G * Lq) one decode CTA handles
 PREFILL_ROWS_PER_CTA = 256
 
@@ -279,14 +279,16 @@ def split_bounds(n: int, num_splits: int) -> List[int]:
 
 
 def auto_num_splits(B: int, Hkv: int, Hq: int, Lq: int, n: int, num_sms: int, D: int = 128) -> int:
-    """Automatic split count: enough CTAs to give every SM CTAS_PER_SM of them
-    (CTAS_PER_SM_D256 for D = 256), no split shorter than SPLIT_MIN_KEYS keys,
-    at most SPLIT_MAX, and no split that the chunk rounding would leave empty.
-    (Reading of "num_splits sized to fill the SMs": the pages give no formula.)"""
+    """Automatic split count: ceil(num_sms * num / den) CTAs in all, with
+    (num, den) = CTAS_PER_SM (CTAS_PER_SM_D256 for D = 256), no split shorter
+    than SPLIT_MIN_KEYS keys, at most SPLIT_MAX, and no split that the chunk
+    rounding would leave empty.  (Reading of "num_splits sized to fill the
+    SMs": the pages give no formula.)"""
     G = Hq // Hkv
     row_groups = _ceil_div(G * Lq, DECODE_ROWS_PER_CTA)
     units = B * Hkv * row_groups
-    target = (CTAS_PER_SM_D256 if D > 128 else CTAS_PER_SM) * num_sms
+    num, den = CTAS_PER_SM_D256 if D > 128 else CTAS_PER_SM
+    target = _ceil_div(num_sms * num, den)
     s = max(1, _ceil_div(target, max(units, 1)))
     s = min(s, max(1, _ceil_div(n, SPLIT_MIN_KEYS)), SPLIT_MAX)
     if n > 0:

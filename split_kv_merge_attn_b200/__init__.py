@@ -12,7 +12,7 @@ Entry points (same names as the C ABI):
 * ``attn_fwd_lse``        prefill / varlen attention, O and per-row log2 LSE
 * ``attn_splitkv_decode`` split-KV decode (stable per-split online softmax)
 * ``merge_state``         merge partial (O, LSE) pairs of disjoint KV ranges
-* ``attn_splitkv_plan``, ``attn_splitkv_workspace``, ``attn_fwd_lse_workspace``,
+* ``attn_splitkv_plan``, ``attn_splitkv_workspace``, ``attn_splitkv_workspace_init``, ``attn_fwd_lse_workspace``,
   ``attn_varlen_plan``     host-side planning / sizing queries
 """
 from __future__ import annotations
@@ -41,6 +41,9 @@ SIGNATURES = {
                                             _c_float, _c_int, _vp, _c_int, _vp]),
     "attn_splitkv_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "attn_splitkv_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "attn_splitkv_decode_fused": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                           _c_float, _c_int, _vp, _c_int, _vp, _c_size, _vp]),
+    "attn_splitkv_workspace_init": (_c_int, [_vp, _c_size, _vp]),
     "merge_state": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                              _c_i64, _c_i64, _vp]),
     "skv_status_string": (ctypes.c_char_p, [_c_int]),
@@ -233,10 +236,22 @@ def attn_fwd_lse(q, k, v, scale: Optional[float] = None, layout: str = "HND", cu
     return out, lse
 
 
+def attn_splitkv_workspace_init(workspace, stream=None):
+    """Zeroes a decode workspace (uint8 device tensor) on `stream`: needed once
+    before its first use by attn_splitkv_decode(..., fused=True)."""
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().attn_splitkv_workspace_init(_ptr(workspace), nbytes, _stream(stream, workspace.device)),
+           "attn_splitkv_workspace_init")
+    return workspace
+
+
 def attn_splitkv_decode(q, k, v, scale: Optional[float] = None, kv_len=None, num_splits: int = 0, out=None,
-                        lse=None, return_lse: bool = True, workspace=None, stream=None):
+                        lse=None, return_lse: bool = True, workspace=None, stream=None, fused: bool = False):
     """Split-KV decode: q [B,Hq,Lq,D], k/v [B,Hkv,Lkv,D] (HND).  kv_len: optional
-    int32 device tensor [B].  num_splits 0 = automatic.  Returns (out, lse)."""
+    int32 device tensor [B].  num_splits 0 = automatic.  Returns (out, lse).
+    fused=True: one kernel launch, the splits merged by the last CTA of each
+    group (attn_splitkv_decode_fused); a workspace passed in must have been
+    zeroed once (attn_splitkv_workspace_init), one allocated here is zeroed."""
     torch = _torch()
     _need_cuda(q, k, v, out, lse, kv_len)
     B, Hq, Lq, D = q.shape
@@ -254,11 +269,14 @@ def attn_splitkv_decode(q, k, v, scale: Optional[float] = None, kv_len=None, num
         sms = torch.cuda.get_device_properties(q.device).multi_processor_count
         splits, _ = attn_splitkv_plan(B, Hq, Hkv, Lq, Lkv, D, sms, 0)
     nbytes = attn_splitkv_workspace(B, Hq, Lq, D, splits)
+    fresh = workspace is None and nbytes > 0
     workspace, wbytes = _workspace(nbytes, q.device, workspace)
-    st = lib().attn_splitkv_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lkv, D,
-                                   float(scale), _dtype_code(q), _ptr(kv_len), int(splits), _ptr(workspace),
-                                   wbytes, _stream(stream, q.device))
-    _check(st, "attn_splitkv_decode")
+    if fused and fresh:
+        attn_splitkv_workspace_init(workspace, stream)
+    fn = lib().attn_splitkv_decode_fused if fused else lib().attn_splitkv_decode
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lkv, D, float(scale), _dtype_code(q),
+            _ptr(kv_len), int(splits), _ptr(workspace), wbytes, _stream(stream, q.device))
+    _check(st, "attn_splitkv_decode_fused" if fused else "attn_splitkv_decode")
     return out, lse
 
 

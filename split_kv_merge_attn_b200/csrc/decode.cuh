@@ -4,9 +4,12 @@
 // Prior art: the ExecuTorch split-K decode kernels (PR #22133, "Prevent
 // Voxtral NaNs in CUDA split-K attention").  That PR replaced a fixed
 // exponent offset by a per-split running max with rescaled partials; this
-// kernel does the same (stable online softmax in the exp2 domain), writes
-// every partial slot (empty splits write O = 0, LSE = -inf) and leaves the
-// cross-split reduction to the merge_state kernel.
+// kernel does the same (stable online softmax in the exp2 domain) and writes
+// every partial slot (empty splits write O = 0, LSE = -inf).  The cross-split
+// reduction is either the merge_state kernel, launched after it, or done in
+// this launch: with an arrival counter per (batch, kv head, row group), the
+// CTA that finishes last among the group's splits merges their partials
+// itself (no CTA ever waits for another) and sets the counter back to zero.
 //
 // B200 mapping:
 //  * the G*Lq query rows that share one kv head (GQA) form one 16-row M tile,
@@ -30,6 +33,8 @@ constexpr int kDecodeKeysPerTile = 64;
 constexpr int kDecodeRows = 16;
 constexpr int kDecodeConsumerWarps = 4;
 constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
+constexpr int kSplitMaxDevice = 256;   // largest num_splits (the host planner's cap)
+constexpr int kMergeStageOffset = kSplitMaxDevice * kDecodeRows * 4 + 128;  // after weights + 1/sum
 
 template <int D>
 struct DecodeCfg {
@@ -52,12 +57,186 @@ struct DecodeArgs {
   float* lse;
   float* part_o;
   float* part_lse;
+  int* counters;  // [grid.y] arrival counters (zero between calls), or null: merge_state merges
   const int* kv_len;
   int B, Hq, Hkv, Lq, Lkv;
   int num_splits;
   int row_groups;
   float scale_log2;
 };
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// Merge of every split's partial (O, LSE) of one row group, run by the 128
+// consumer threads of the CTA that finished last; `smem` is the (idle) K/V
+// ring.  Per row: M = max_s L_s, w_s = 2^(L_s - M) (0 for -inf),
+// O = sum_s w_s O_s / sum_s w_s, LSE = M + log2(sum_s w_s); all splits empty
+// gives O = 0, LSE = -inf.  The partials of a row group are contiguous
+// (rn rows x D floats per split); they are staged into shared memory with
+// 16-byte cp.async copies (L2 only), as many splits per batch as fit.
+template <int D, typename T>
+__device__ __forceinline__ void decode_merge_group(const DecodeArgs& a, uint8_t* smem, int smem_bytes,
+                                                   int64_t orow0, int rn, int64_t rows_all) {
+  constexpr int kV = D / 4;                  // float4 per row
+  constexpr int kJ = kDecodeRows * kV / 128; // float4 outputs per thread (at most)
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = a.num_splits;
+  float* wt = reinterpret_cast<float*>(smem);  // [S][16] weights
+  float* rinv = wt + kSplitMaxDevice * kDecodeRows;  // [16] 1 / sum of weights
+  float4* stage = reinterpret_cast<float4*>(smem + kMergeStageOffset);
+  const int nv = rn * kV;
+  const int cap = (smem_bytes - kMergeStageOffset) / 16;
+  const int nb = max(1, cap / nv);  // splits per batch
+
+  const float4* po = reinterpret_cast<const float4*>(a.part_o);
+  const uint32_t stage_addr = smem_u32(stage);
+  // copies of splits [s0, s1) into the staging area (one commit group)
+  auto issue = [&](int s0, int s1) {
+    for (int s = s0; s < s1; ++s) {
+      const float4* src = po + (s * rows_all + orow0) * kV;
+#pragma unroll
+      for (int j = 0; j < kJ; ++j) {
+        const int v = tid + 128 * j;
+        if (v < nv) cp_async_16(stage_addr + static_cast<uint32_t>(((s - s0) * nv + v) * 16), src + v);
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  issue(0, min(S, nb));  // the first batch is in flight while the weights are computed
+
+  // ---- weights: warp w takes rows w, w+4, ...
+  for (int r = warp; r < rn; r += kDecodeConsumerWarps) {
+    float L[kSplitMaxDevice / 32];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kSplitMaxDevice / 32; ++i) {
+      const int s = lane + 32 * i;
+      L[i] = (s < S) ? __ldcg(a.part_lse + s * rows_all + orow0 + r) : -INFINITY;
+      mx = fmaxf(mx, L[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSplitMaxDevice / 32; ++i) {
+      const int s = lane + 32 * i;
+      const float w = (L[i] == -INFINITY) ? 0.f : ex2_approx(L[i] - mx);
+      if (s < S) wt[s * kDecodeRows + r] = w;
+      sum += w;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) {
+      rinv[r] = sum > 0.f ? 1.0f / sum : 0.f;
+      if (a.lse != nullptr) a.lse[orow0 + r] = sum > 0.f ? mx + __log2f(sum) : -INFINITY;
+    }
+  }
+  named_barrier_sync(1, kDecodeConsumerWarps * 32);
+
+  // ---- O: thread t owns float4 outputs t, t + 128, ...
+  float4 acc[kJ];
+#pragma unroll
+  for (int j = 0; j < kJ; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < S; s0 += nb) {
+    const int s1 = min(S, s0 + nb);
+    if (s0 > 0) issue(s0, s1);
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    // each thread reads back only the slots it copied itself
+    for (int s = s0; s < s1; ++s) {
+#pragma unroll
+      for (int j = 0; j < kJ; ++j) {
+        const int v = tid + 128 * j;
+        if (v < nv) {
+          const float w = wt[s * kDecodeRows + v / kV];
+          const float4 x = stage[(s - s0) * nv + v];
+          acc[j].x = fmaf(w, x.x, acc[j].x);
+          acc[j].y = fmaf(w, x.y, acc[j].y);
+          acc[j].z = fmaf(w, x.z, acc[j].z);
+          acc[j].w = fmaf(w, x.w, acc[j].w);
+        }
+      }
+    }
+  }
+  T* out = static_cast<T*>(a.out) + orow0 * D;
+#pragma unroll
+  for (int j = 0; j < kJ; ++j) {
+    const int v = tid + 128 * j;
+    if (v < nv) {
+      const float inv = rinv[v / kV];
+      uint2 u;
+      u.x = pack2<T>(acc[j].x * inv, acc[j].y * inv);
+      u.y = pack2<T>(acc[j].z * inv, acc[j].w * inv);
+      *reinterpret_cast<uint2*>(out + static_cast<int64_t>(v) * 4) = u;
+    }
+  }
+}
+
+// Final (one split) or partial (split > 1) result of rows r of this CTA's
+// group from the four consumer warps' states; 8 threads per row, each a D/8
+// slice.
+template <int D, typename T>
+__device__ __forceinline__ void decode_write_rows(const DecodeArgs& a, const float* cm, const float* cl,
+                                                  const float* co, int b, int hkv, int G, int rglob, int r, int sl,
+                                                  int split) {
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kDecodeConsumerWarps; ++w) M = fmaxf(M, cm[w * 16 + r]);
+  float e[kDecodeConsumerWarps];
+  float L = 0.f;
+#pragma unroll
+  for (int w = 0; w < kDecodeConsumerWarps; ++w) {
+    const float mw = cm[w * 16 + r];
+    e[w] = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
+    L += e[w] * cl[w * 16 + r];
+  }
+  const float inv = (L > 0.f) ? 1.0f / L : 0.f;
+  const float lse_val = (L > 0.f) ? M + __log2f(L) : -INFINITY;
+  const int h = hkv * G + rglob / a.Lq;
+  const int i = rglob % a.Lq;
+  const int64_t orow = (static_cast<int64_t>(b) * a.Hq + h) * a.Lq + i;
+  const int64_t rows_all = static_cast<int64_t>(a.B) * a.Hq * a.Lq;
+  constexpr int per = D / 8;
+  if (a.num_splits == 1) {
+    T* dst = static_cast<T*>(a.out) + orow * D + sl * per;
+#pragma unroll
+    for (int c = 0; c < per; c += 8) {
+      float v[8];
+#pragma unroll
+      for (int q2 = 0; q2 < 8; ++q2) {
+        const int d = sl * per + c + q2;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecodeConsumerWarps; ++w) acc = fmaf(e[w], co[(w * 16 + r) * D + d], acc);
+        v[q2] = acc * inv;
+      }
+      uint4 u;
+      u.x = pack2<T>(v[0], v[1]);
+      u.y = pack2<T>(v[2], v[3]);
+      u.z = pack2<T>(v[4], v[5]);
+      u.w = pack2<T>(v[6], v[7]);
+      *reinterpret_cast<uint4*>(dst + c) = u;
+    }
+    if (sl == 0 && a.lse != nullptr) a.lse[orow] = lse_val;
+  } else {
+    float* dst = a.part_o + (static_cast<int64_t>(split) * rows_all + orow) * D + sl * per;
+#pragma unroll
+    for (int c = 0; c < per; c += 4) {
+      float v[4];
+#pragma unroll
+      for (int q2 = 0; q2 < 4; ++q2) {
+        const int d = sl * per + c + q2;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecodeConsumerWarps; ++w) acc = fmaf(e[w], co[(w * 16 + r) * D + d], acc);
+        v[q2] = acc * inv;
+      }
+      *reinterpret_cast<float4*>(dst + c) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+    if (sl == 0) a.part_lse[static_cast<int64_t>(split) * rows_all + orow] = lse_val;
+  }
+}
 
 template <int D, typename T>
 __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -286,7 +465,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
 
   // ---- combine the four warps' states
   named_barrier_sync(1, kDecodeConsumerWarps * 32);
-  if (!ok || *abort_flag) return;
+  (void)ok;  // a failed wait has set the abort flag, which every consumer thread sees after the barrier
+  const bool aborted = *abort_flag != 0;
+  if (aborted && (a.counters == nullptr || a.num_splits == 1)) return;
   lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], 1);
   lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], 2);
   lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], 1);
@@ -312,63 +493,29 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
   const int r = tid >> 3;
   const int sl = tid & 7;
   const int rglob = rg * kDecodeRows + r;
-  if (rglob >= rows_total) return;
-  float M = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < kDecodeConsumerWarps; ++w) M = fmaxf(M, cm[w * 16 + r]);
-  float e[kDecodeConsumerWarps];
-  float L = 0.f;
-#pragma unroll
-  for (int w = 0; w < kDecodeConsumerWarps; ++w) {
-    const float mw = cm[w * 16 + r];
-    e[w] = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
-    L += e[w] * cl[w * 16 + r];
+  if (!aborted && rglob < rows_total) decode_write_rows<D, T>(a, cm, cl, co, b, hkv, G, rglob, r, sl, split);
+  if (a.counters == nullptr || a.num_splits == 1) return;
+
+  // ---- in-launch merge: the last CTA of this row group to arrive merges.
+  // The barrier orders every consumer thread's partial stores before thread
+  // 0's arrival, whose release (cumulative) publishes them; its acquire, with
+  // the next barrier, orders the last CTA's loads after every other split's
+  // release.
+  named_barrier_sync(1, kDecodeConsumerWarps * 32);
+  volatile int* last_flag = abort_flag + 1;
+  if (tid == 0) {
+    int old;
+    asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], 1;" : "=r"(old) : "l"(a.counters + blockIdx.y) : "memory");
+    if (old < 0 || old >= a.num_splits) record_error(kErrDecodeCounter);  // counter was not zero before the call
+    *last_flag = (old == a.num_splits - 1) ? 1 : 0;
   }
-  const float inv = (L > 0.f) ? 1.0f / L : 0.f;
-  const float lse_val = (L > 0.f) ? M + __log2f(L) : -INFINITY;
-  const int h = hkv * G + rglob / a.Lq;
-  const int i = rglob % a.Lq;
-  const int64_t orow = (static_cast<int64_t>(b) * a.Hq + h) * a.Lq + i;
-  const int64_t rows_all = static_cast<int64_t>(a.B) * a.Hq * a.Lq;
-  constexpr int per = D / 8;
-  if (a.num_splits == 1) {
-    T* dst = static_cast<T*>(a.out) + orow * D + sl * per;
-#pragma unroll
-    for (int c = 0; c < per; c += 8) {
-      float v[8];
-#pragma unroll
-      for (int q2 = 0; q2 < 8; ++q2) {
-        const int d = sl * per + c + q2;
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecodeConsumerWarps; ++w) acc = fmaf(e[w], co[(w * 16 + r) * D + d], acc);
-        v[q2] = acc * inv;
-      }
-      uint4 u;
-      u.x = pack2<T>(v[0], v[1]);
-      u.y = pack2<T>(v[2], v[3]);
-      u.z = pack2<T>(v[4], v[5]);
-      u.w = pack2<T>(v[6], v[7]);
-      *reinterpret_cast<uint4*>(dst + c) = u;
-    }
-    if (sl == 0 && a.lse != nullptr) a.lse[orow] = lse_val;
-  } else {
-    float* dst = a.part_o + (static_cast<int64_t>(split) * rows_all + orow) * D + sl * per;
-#pragma unroll
-    for (int c = 0; c < per; c += 4) {
-      float v[4];
-#pragma unroll
-      for (int q2 = 0; q2 < 4; ++q2) {
-        const int d = sl * per + c + q2;
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecodeConsumerWarps; ++w) acc = fmaf(e[w], co[(w * 16 + r) * D + d], acc);
-        v[q2] = acc * inv;
-      }
-      *reinterpret_cast<float4*>(dst + c) = make_float4(v[0], v[1], v[2], v[3]);
-    }
-    if (sl == 0) a.part_lse[static_cast<int64_t>(split) * rows_all + orow] = lse_val;
-  }
+  named_barrier_sync(1, kDecodeConsumerWarps * 32);
+  if (*last_flag == 0) return;
+  const int64_t orow0 = (static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(hkv) * G) * a.Lq +
+                        static_cast<int64_t>(rg) * kDecodeRows;
+  decode_merge_group<D, T>(a, ring, Cfg::kRingBytes, orow0, min(kDecodeRows, rows_total - rg * kDecodeRows),
+                           static_cast<int64_t>(a.B) * a.Hq * a.Lq);
+  if (tid == 0) a.counters[blockIdx.y] = 0;  // ready for the next call on this workspace
 }
 
 }  // namespace skv

@@ -56,10 +56,25 @@ FwdWorkspace fwd_workspace(int B, int Hkv, int Sk, int D, skv_layout layout, int
   return w;
 }
 
-size_t decode_workspace(int B, int Hq, int Lq, int D, int splits) {
-  if (splits <= 1) return 0;
+// [splits][rows][D] fp32 partial O | [splits][rows] fp32 partial LSE |
+// [rows] int32 arrival counters (one per (batch, kv head, row group) are used;
+// rows bounds their number), each region 256-byte aligned.
+struct DecodeWs {
+  size_t part_o = 0, part_lse = 0, counters = 0, total = 0;
+};
+DecodeWs decode_ws_layout(int B, int Hq, int Lq, int D, int splits) {
+  DecodeWs w;
+  if (splits <= 1) return w;
   const size_t rows = static_cast<size_t>(B) * Hq * Lq;
-  return skv::align256(static_cast<size_t>(splits) * rows * D * 4) + skv::align256(static_cast<size_t>(splits) * rows * 4);
+  w.part_o = 0;
+  w.part_lse = skv::align256(static_cast<size_t>(splits) * rows * D * 4);
+  w.counters = w.part_lse + skv::align256(static_cast<size_t>(splits) * rows * 4);
+  w.total = w.counters + skv::align256(rows * 4);
+  return w;
+}
+
+size_t decode_workspace(int B, int Hq, int Lq, int D, int splits) {
+  return decode_ws_layout(B, Hq, Lq, D, splits).total;
 }
 
 }  // namespace
@@ -103,7 +118,9 @@ skv_status attn_splitkv_plan(int B, int Hq, int Hkv, int Lq, int n, int D, int n
     const int64_t G = Hq / Hkv;
     const int64_t row_groups = skv::ceil_div64(G * Lq, skv::kDecodeRowsPerCta);
     const int64_t units = static_cast<int64_t>(B) * Hkv * row_groups;
-    const int64_t target = static_cast<int64_t>(D > 128 ? skv::kCtasPerSmD256 : skv::kCtasPerSm) * num_sms;
+    const int64_t num = D > 128 ? skv::kCtasPerSmD256Num : skv::kCtasPerSmNum;
+    const int64_t den = D > 128 ? skv::kCtasPerSmD256Den : skv::kCtasPerSmDen;
+    const int64_t target = skv::ceil_div64(static_cast<int64_t>(num_sms) * num, den);
     int64_t ss = std::max<int64_t>(1, skv::ceil_div64(target, units));
     ss = std::min<int64_t>(ss, std::max<int64_t>(1, skv::ceil_div64(n, skv::kSplitMinKeys)));
     ss = std::min<int64_t>(ss, skv::kSplitMax);
@@ -245,9 +262,10 @@ skv_status attn_fwd_lse(const void* q, const void* k, const void* v, void* out, 
 
 // ------------------------------------------------------------------ decode
 
-skv_status attn_splitkv_decode(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
-                               int Hkv, int Lq, int Lkv, int D, float scale, skv_dtype dtype, const int32_t* kv_len,
-                               int num_splits, void* workspace, size_t workspace_bytes, skv_stream_t stream) {
+namespace {
+skv_status decode_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                       int Lq, int Lkv, int D, float scale, skv_dtype dtype, const int32_t* kv_len, int num_splits,
+                       void* workspace, size_t workspace_bytes, skv_stream_t stream, bool in_launch_merge) {
   if (q == nullptr || out == nullptr) return SKV_ERR_INVALID_ARG;
   if ((k == nullptr || v == nullptr) && Lkv != 0) return SKV_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return SKV_ERR_INVALID_ARG;
@@ -275,22 +293,47 @@ skv_status attn_splitkv_decode(const void* q, const void* k, const void* v, void
   if (need > 0 && (workspace == nullptr || !aligned(workspace, 256))) return SKV_ERR_INVALID_ARG;
   float* part_o = nullptr;
   float* part_lse = nullptr;
+  int* counters = nullptr;
   if (splits > 1) {
-    const size_t rows = static_cast<size_t>(B) * Hq * Lq;
-    part_o = static_cast<float*>(workspace);
-    part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                        skv::align256(static_cast<size_t>(splits) * rows * D * 4));
+    const DecodeWs w = decode_ws_layout(B, Hq, Lq, D, splits);
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    part_o = reinterpret_cast<float*>(wsb + w.part_o);
+    part_lse = reinterpret_cast<float*>(wsb + w.part_lse);
+    if (in_launch_merge) counters = reinterpret_cast<int*>(wsb + w.counters);
   }
-  int e = skv::launch_decode(q, k, v, out, lse, part_o, part_lse, kv_len, B, Hq, Hkv, Lq, Lkv, D, scale, dtype, splits,
-                             stream);
+  int e = skv::launch_decode(q, k, v, out, lse, part_o, part_lse, counters, kv_len, B, Hq, Hkv, Lq, Lkv, D, scale,
+                             dtype, splits, stream);
   if (e) return cuda_status(e);
-  if (splits > 1) {
+  if (splits > 1 && !in_launch_merge) {
     const int64_t rows = static_cast<int64_t>(B) * Hq * Lq;
     e = skv::launch_merge_state(part_o, part_lse, out, lse, splits, 1, 1, static_cast<int>(rows), D, 0, SKV_FP32,
                                 dtype, rows * D, rows, stream, /*dependent=*/true);
     if (e) return cuda_status(e);
   }
   return SKV_OK;
+}
+
+}  // namespace
+
+skv_status attn_splitkv_decode(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                               int Hkv, int Lq, int Lkv, int D, float scale, skv_dtype dtype, const int32_t* kv_len,
+                               int num_splits, void* workspace, size_t workspace_bytes, skv_stream_t stream) {
+  return decode_impl(q, k, v, out, lse, B, Hq, Hkv, Lq, Lkv, D, scale, dtype, kv_len, num_splits, workspace,
+                     workspace_bytes, stream, /*in_launch_merge=*/false);
+}
+
+skv_status attn_splitkv_decode_fused(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                                     int Hq, int Hkv, int Lq, int Lkv, int D, float scale, skv_dtype dtype,
+                                     const int32_t* kv_len, int num_splits, void* workspace, size_t workspace_bytes,
+                                     skv_stream_t stream) {
+  return decode_impl(q, k, v, out, lse, B, Hq, Hkv, Lq, Lkv, D, scale, dtype, kv_len, num_splits, workspace,
+                     workspace_bytes, stream, /*in_launch_merge=*/true);
+}
+
+skv_status attn_splitkv_workspace_init(void* workspace, size_t workspace_bytes, skv_stream_t stream) {
+  if (workspace_bytes == 0) return SKV_OK;
+  if (workspace == nullptr) return SKV_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 // ------------------------------------------------------------------ merge

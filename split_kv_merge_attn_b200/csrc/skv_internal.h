@@ -15,6 +15,7 @@ namespace skv {
 enum DeviceError : int {
   kErrDecodeEmptyWait = 0x101,
   kErrDecodeFullWait = 0x102,
+  kErrDecodeCounter = 0x103,   // a decode arrival counter was not zero before the call
   kErrPrefillWait = 0x201,
 };
 
@@ -22,8 +23,12 @@ enum DeviceError : int {
 constexpr int kSplitAlign = 64;
 constexpr int kSplitMinKeys = 128;
 constexpr int kSplitMax = 256;
-constexpr int kCtasPerSm = 2;       // decode CTAs resident per SM, D <= 128
-constexpr int kCtasPerSmD256 = 1;   // and for D = 256
+// The automatic decode plan aims for ceil(num_sms * num / den) CTAs in all:
+// one per SM for D <= 128 (the kernel could hold two, but fewer, longer splits
+// measured faster: fewer concurrent K/V streams and a smaller merge) and two
+// per three SMs for D = 256, whose CTA keeps twice the bytes in flight.
+constexpr int kCtasPerSmNum = 1, kCtasPerSmDen = 1;
+constexpr int kCtasPerSmD256Num = 2, kCtasPerSmD256Den = 3;
 constexpr int kDecodeRowsPerCta = 16;
 constexpr int kPrefillRowsPerCta = 256;
 
@@ -38,9 +43,11 @@ int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, f
                        int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream,
                        bool dependent = false);
 
+// counters: null = partials only (merge_state merges them); else per-group
+// arrival counters, zero on entry, and the last CTA of each group merges.
 int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, float* part_o,
-                  float* part_lse, const int32_t* kv_len, int B, int Hq, int Hkv, int Lq, int Lkv, int D,
-                  float scale, skv_dtype dt, int num_splits, skv_stream_t stream);
+                  float* part_lse, int* counters, const int32_t* kv_len, int B, int Hq, int Hkv, int Lq, int Lkv,
+                  int D, float scale, skv_dtype dt, int num_splits, skv_stream_t stream);
 
 struct PrefillLaunch {
   const void* q;

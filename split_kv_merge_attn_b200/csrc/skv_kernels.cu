@@ -189,8 +189,8 @@ int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeAr
 }  // namespace
 
 int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, float* part_o,
-                  float* part_lse, const int32_t* kv_len, int B, int Hq, int Hkv, int Lq, int Lkv, int D,
-                  float scale, skv_dtype dt, int num_splits, skv_stream_t stream) {
+                  float* part_lse, int* counters, const int32_t* kv_len, int B, int Hq, int Hkv, int Lq, int Lkv,
+                  int D, float scale, skv_dtype dt, int num_splits, skv_stream_t stream) {
   const int G = Hq / Hkv;
   DecodeArgs a;
   a.q = q;
@@ -198,6 +198,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
   a.lse = lse;
   a.part_o = part_o;
   a.part_lse = part_lse;
+  a.counters = counters;
   a.kv_len = kv_len;
   a.B = B;
   a.Hq = Hq;

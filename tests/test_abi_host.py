@@ -112,11 +112,36 @@ def test_attn_splitkv_decode_rejects_invalid_arguments():
     assert dec(splits=8, ws=None, wsb=need) == INVALID
 
 
+def dec_fused(**kw):
+    a = dict(q=P16, k=P16, v=P16, out=P16, lse=None, B=1, Hq=32, Hkv=8, Lq=1, Lkv=4096, D=128, scale=0.1, dt=0,
+             kv_len=None, splits=1, ws=None, wsb=0)
+    a.update(kw)
+    return skv.lib().attn_splitkv_decode_fused(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"],
+                                               a["Hkv"], a["Lq"], a["Lkv"], a["D"], a["scale"], a["dt"], a["kv_len"],
+                                               a["splits"], a["ws"], a["wsb"], None)
+
+
+def test_attn_splitkv_decode_fused_validates_like_the_two_kernel_decode():
+    assert dec_fused(q=None) == INVALID
+    assert dec_fused(Hq=30) == INVALID
+    assert dec_fused(splits=257) == INVALID
+    assert dec_fused(D=96) == UNSUPPORTED
+    need = skv.attn_splitkv_workspace(1, 32, 1, 128, 8)
+    assert dec_fused(splits=8, ws=P16, wsb=need - 1) == WS_SMALL
+    assert dec_fused(splits=8, ws=None, wsb=need) == INVALID
+
+
+def test_workspace_init_arguments():
+    assert skv.lib().attn_splitkv_workspace_init(None, 0, None) == skv.SKV_OK
+    assert skv.lib().attn_splitkv_workspace_init(None, 256, None) == INVALID
+
+
 def O_ws(B, Hq, Lq, D, S):
-    """Workspace of S splits: fp32 partial O then fp32 partial LSE, each 256-byte aligned."""
+    """Workspace of S splits: fp32 partial O, fp32 partial LSE, then one int32
+    arrival counter per row (the fused decode's), each 256-byte aligned."""
     a = lambda x: (x + 255) // 256 * 256
     rows = B * Hq * Lq
-    return a(S * rows * D * 4) + a(S * rows * 4) if S > 1 else 0
+    return a(S * rows * D * 4) + a(S * rows * 4) + a(rows * 4) if S > 1 else 0
 
 
 def test_decode_workspace_sizes():

@@ -419,21 +419,25 @@ def test_split_bounds_partition():
 
 
 def test_split_plan_hand_values():
-    # Lkv = 32768 over 8 kv heads on 148 SMs: ceil(296 / 8) = 37 splits,
-    # C = roundup(ceil(32768/37)=886, 64) = 896, ceil(32768/896) = 37
-    assert O.auto_num_splits(1, 8, 32, 1, 32768, 148) == 37
-    assert O.split_bounds(32768, 37)[1] == 896
-    assert O.split_bounds(32768, 37)[-2] == 36 * 896
-    # Lkv = 4096: 37 capped to ceil(4096/128) = 32; C = 128 -> 32 splits
-    assert O.auto_num_splits(1, 8, 32, 1, 4096, 148) == 32
-    # D=128 rule on a 4-kv-head shape (G*Lq = 16): ceil(296/4) = 74, Lkv 16384 -> C = 256 -> 64
-    assert O.auto_num_splits(1, 4, 16, 4, 16384, 148) == 64
-    # G*Lq = 32 rows -> two row groups per kv head
-    assert O.auto_num_splits(1, 4, 16, 8, 16384, 148) == 37
-    # D = 256 aims at one CTA per SM: ceil(148/4) = 37, C = roundup(443, 64) = 448 -> 37
-    assert O.auto_num_splits(1, 4, 16, 4, 16384, 148, D=256) == 37
-    # two row groups: ceil(148/8) = 19, C = roundup(863, 64) = 896 -> ceil(16384/896) = 19
-    assert O.auto_num_splits(1, 4, 16, 8, 16384, 148, D=256) == 19
+    # Lkv = 32768 over 8 kv heads on 148 SMs (one CTA per SM): ceil(148 / 8) = 19
+    # splits, C = roundup(ceil(32768/19)=1725, 64) = 1728, ceil(32768/1728) = 19,
+    # the last split holding 32768 - 18 * 1728 = 1664 keys
+    assert O.auto_num_splits(1, 8, 32, 1, 32768, 148) == 19
+    assert O.split_bounds(32768, 19)[1] == 1728
+    assert O.split_bounds(32768, 19)[-2] == 18 * 1728
+    # Lkv = 4096: C = roundup(ceil(4096/19)=216, 64) = 256 -> 16 splits
+    assert O.auto_num_splits(1, 8, 32, 1, 4096, 148) == 16
+    # a 4-kv-head shape (G*Lq = 16): ceil(148/4) = 37, Lkv 16384 -> C = roundup(443, 64) = 448 -> 37
+    assert O.auto_num_splits(1, 4, 16, 4, 16384, 148) == 37
+    # G*Lq = 32 rows -> two row groups per kv head: ceil(148/8) = 19, C = 896 -> 19
+    assert O.auto_num_splits(1, 4, 16, 8, 16384, 148) == 19
+    # D = 256 aims at two CTAs per three SMs: ceil(296/3) = 99, ceil(99/4) = 25,
+    # C = roundup(ceil(16384/25)=656, 64) = 704 -> ceil(16384/704) = 24
+    assert O.auto_num_splits(1, 4, 16, 4, 16384, 148, D=256) == 24
+    # and Lkv = 32768: C = roundup(1311, 64) = 1344 -> ceil(32768/1344) = 25
+    assert O.auto_num_splits(1, 4, 16, 4, 32768, 148, D=256) == 25
+    # two row groups: ceil(99/8) = 13, C = roundup(1261, 64) = 1280 -> 13
+    assert O.auto_num_splits(1, 4, 16, 8, 16384, 148, D=256) == 13
     assert O.auto_num_splits(1, 8, 32, 1, 0, 148) == 1
     assert O.auto_num_splits(1, 8, 32, 1, 100, 148) == 1
 
