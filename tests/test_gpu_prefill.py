@@ -128,6 +128,32 @@ def test_dense_increasing_logits_force_rescales():
     check_lse(lse, l_ref)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_dense_max_jumps_inside_tiles(dtype):
+    """Planted keys raise the running max by far more than the lazy-rescale
+    threshold at chosen places: in the second half of a 128-key tile (its first
+    half already published to the PV products), in the first half of a later
+    tile, and in a tile's last key.  Even rows see the jumps, odd rows see the
+    same keys as large negative logits, so warps mix rows that rescale with
+    rows that do not."""
+    B, H, Sq, Sk, D = 1, 2, 256, 1024, 128
+    d = W.dense_case(B, H, H, Sq, Sk, D, seed=12, dtype=dtype)
+    scale = d["scale"]
+    q = d["q"].float()
+    k = d["k"].float()
+    sign = torch.tensor([4.0, -4.0]).repeat(Sq // 2)
+    q[:, :, :, 0] = sign                              # q . e0 = +-4
+    for pos, logit in [(3 * 128 + 64 + 7, 20.0), (5 * 128 + 3, 40.0), (6 * 128 + 100, 60.0), (7 * 128 + 127, 75.0)]:
+        k[:, :, pos, :] = 0.0
+        k[:, :, pos, 0] = logit / (4.0 * scale)       # natural-log logit +-logit
+    t = d["q"].dtype
+    d["q"], d["k"] = q.to(t), k.to(t)
+    out, lse = run_dense(d)
+    o_ref, l_ref = O.dense(d["q"], d["k"], d["v"], d["scale"])
+    check_o(out, o_ref, vmax(d["v"]))
+    check_lse(lse, l_ref)
+
+
 # ------------------------------------------------------------ varlen
 
 def test_varlen_small_ragged():
