@@ -38,6 +38,7 @@ __all__ = [
     "to_f64", "attention_rows", "dense", "varlen", "decode", "merge",
     "kv_mean", "smooth_shift", "smoothed_attention_rows", "chunked",
     "split_bounds", "auto_num_splits", "varlen_schedule", "lse_varlen_to_dense",
+    "causal_key_counts",
 ]
 
 
@@ -52,19 +53,32 @@ def to_f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float
-                   ) -> Tuple[np.ndarray, np.ndarray]:
+def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                   key_counts: Optional[Sequence[int]] = None) -> Tuple[np.ndarray, np.ndarray]:
     """O and log2-LSE for query rows q [n, D] over keys k [m, D], values v [m, D].
 
     Definition: ARK return_lse issue, "Expected:" (one LSE per query row, log2
     units, original logits, LSE = log2(sum_j exp(scale * q . k_j))).  The max is
     subtracted before exponentiating only to keep float64 finite; it cancels
     exactly in both O and LSE.
+
+    key_counts (optional, one per row): row r sees only keys [0, key_counts[r])
+    -- the causal mask, see ``causal_key_counts``.  A row that sees no key gets
+    O = 0 and LSE = -inf, like an empty range.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     n, m = q.shape[0], k.shape[0]
+    if key_counts is not None:
+        o = np.zeros((n, v.shape[1]))
+        lse2 = np.full(n, -np.inf)
+        for r in range(n):
+            c = int(key_counts[r])
+            if c > 0:
+                orow, lrow = attention_rows(q[r:r + 1], k[:c], v[:c], scale)
+                o[r], lse2[r] = orow[0], lrow[0]
+        return o, lse2
     if m == 0:
         return np.zeros((n, v.shape[1])), np.full(n, -np.inf)
     s = scale * (q @ k.T)                       # [n, m] scaled logits
@@ -76,6 +90,20 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float
     return o, lse2
 
 
+def causal_key_counts(n_q: int, n_k: int) -> List[int]:
+    """Keys visible to each query row under the causal mask.
+
+    Not on the pages (they describe only full, non-causal ranges); the plainest
+    adjacent reading, taken for the causal variant: the n_q query rows are the
+    LAST n_q positions of a sequence whose n_k keys are positions 0..n_k-1
+    (bottom-right alignment, as in an autoregressive chunk whose queries follow
+    the cached keys), so row i sees keys j <= i + n_k - n_q, i.e. the first
+    clamp(i + n_k - n_q + 1, 0, n_k) keys.  With n_q = n_k this is the usual
+    lower-triangular mask; rows i < n_q - n_k see no key.
+    """
+    return [min(max(i + n_k - n_q + 1, 0), n_k) for i in range(n_q)]
+
+
 def _hnd(x: np.ndarray, layout: str) -> np.ndarray:
     """View a 4-D array given in ``layout`` as [B, H, S, D]."""
     if layout == "HND":
@@ -85,7 +113,8 @@ def _hnd(x: np.ndarray, layout: str) -> np.ndarray:
     raise ValueError(layout)
 
 
-def dense(q, k, v, scale: float, layout: str = "HND", rows: Optional[Sequence[Tuple[int, int, int]]] = None):
+def dense(q, k, v, scale: float, layout: str = "HND", rows: Optional[Sequence[Tuple[int, int, int]]] = None,
+          causal: bool = False):
     """Dense attention, q [B,Hq,Sq,D] / k,v [B,Hkv,Sk,D] in HND or NHD layout.
 
     Returns (O in the input layout, LSE [B, Hq, Sq]) -- the 3-D dense LSE layout
@@ -96,6 +125,7 @@ def dense(q, k, v, scale: float, layout: str = "HND", rows: Optional[Sequence[Tu
 
     If ``rows`` is given (a list of (b, h, i)), only those query rows are
     computed and (O rows [len, D], LSE [len]) is returned.
+    causal: the mask of ``causal_key_counts`` (per row of each (b, h)).
     """
     q4, k4, v4 = _hnd(to_f64(q), layout), _hnd(to_f64(k), layout), _hnd(to_f64(v), layout)
     B, Hq, Sq, D = q4.shape
@@ -103,24 +133,26 @@ def dense(q, k, v, scale: float, layout: str = "HND", rows: Optional[Sequence[Tu
     if Hq % Hkv != 0:
         raise ValueError("Hq must be a multiple of Hkv")
     G = Hq // Hkv
+    counts = causal_key_counts(Sq, k4.shape[2]) if causal else None
     if rows is not None:
         o_out = np.zeros((len(rows), D))
         l_out = np.zeros(len(rows))
         for r, (b, h, i) in enumerate(rows):
-            o, l = attention_rows(q4[b, h, i:i + 1], k4[b, h // G], v4[b, h // G], scale)
+            kc = None if counts is None else [counts[i]]
+            o, l = attention_rows(q4[b, h, i:i + 1], k4[b, h // G], v4[b, h // G], scale, kc)
             o_out[r], l_out[r] = o[0], l[0]
         return o_out, l_out
     o4 = np.zeros((B, Hq, Sq, D))
     lse = np.zeros((B, Hq, Sq))
     for b in range(B):
         for h in range(Hq):
-            o4[b, h], lse[b, h] = attention_rows(q4[b, h], k4[b, h // G], v4[b, h // G], scale)
+            o4[b, h], lse[b, h] = attention_rows(q4[b, h], k4[b, h // G], v4[b, h // G], scale, counts)
     if layout == "NHD":
         return np.ascontiguousarray(o4.transpose(0, 2, 1, 3)), lse
     return o4, lse
 
 
-def varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float):
+def varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: bool = False):
     """Packed TND attention: q [T, Hq, D], k/v [T_k, Hkv, D].
 
     Sequence b owns query rows [cu_q[b], cu_q[b+1]) and keys
@@ -128,6 +160,7 @@ def varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float):
     global packed row (SGLang sgl_kernel::fwd PR: the varlen path returns
     (num_heads, total_q); the Ascend backend record squeezes [T, H, 1] and
     transposes it to the same [H, T]).
+    causal: the mask of ``causal_key_counts`` within each sequence.
     """
     q3, k3, v3 = to_f64(q), to_f64(k), to_f64(v)
     cq = [int(x) for x in np.asarray(cu_seqlens_q).tolist()]
@@ -139,19 +172,22 @@ def varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float):
     lse = np.full((Hq, T), -np.inf)
     for b in range(len(cq) - 1):
         q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        counts = causal_key_counts(q1 - q0, k1 - k0) if causal else None
         for h in range(Hq):
-            ob, lb = attention_rows(q3[q0:q1, h], k3[k0:k1, h // G], v3[k0:k1, h // G], scale)
+            ob, lb = attention_rows(q3[q0:q1, h], k3[k0:k1, h // G], v3[k0:k1, h // G], scale, counts)
             o[q0:q1, h] = ob
             lse[h, q0:q1] = lb
     return o, lse
 
 
-def decode(q, k, v, scale: float, kv_len: Optional[Sequence[int]] = None):
+def decode(q, k, v, scale: float, kv_len: Optional[Sequence[int]] = None, causal: bool = False):
     """Decode: q [B,Hq,Lq,D], k/v [B,Hkv,Lkv,D] (HND), keys [0, kv_len[b]).
 
     Non-causal: all Lq rows see every key of the range (reading; the pages
     route Lq 2..4 to a split-K kernel without naming a mask).  kv_len=None
     means the full Lkv (ExecuTorch split-K PR, the kv_len docstring).
+    causal: the Lq rows are the last Lq positions, row i sees the first
+    kv_len - Lq + 1 + i keys (``causal_key_counts``; not on the pages).
     Returns (O [B,Hq,Lq,D], LSE [B,Hq,Lq]).
     """
     q4, k4, v4 = to_f64(q), to_f64(k), to_f64(v)
@@ -162,8 +198,9 @@ def decode(q, k, v, scale: float, kv_len: Optional[Sequence[int]] = None):
     lse = np.zeros((B, Hq, Lq))
     for b in range(B):
         n = Lkv if kv_len is None else int(kv_len[b])
+        counts = causal_key_counts(Lq, n) if causal else None
         for h in range(Hq):
-            o[b, h], lse[b, h] = attention_rows(q4[b, h], k4[b, h // G, :n], v4[b, h // G, :n], scale)
+            o[b, h], lse[b, h] = attention_rows(q4[b, h], k4[b, h // G, :n], v4[b, h // G, :n], scale, counts)
     return o, lse
 
 

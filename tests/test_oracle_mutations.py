@@ -12,28 +12,41 @@ _orig_rows = O.attention_rows
 _orig_merge = O.merge
 
 
-def _rows_natural_log(q, k, v, scale):
-    o, l = _orig_rows(q, k, v, scale)
+def _rows_natural_log(q, k, v, scale, key_counts=None):
+    o, l = _orig_rows(q, k, v, scale, key_counts)
     return o, l * math.log(2.0)                    # LSE left in natural units
 
 
-def _rows_no_scale(q, k, v, scale):
-    return _orig_rows(q, k, v, 1.0)
+def _rows_no_scale(q, k, v, scale, key_counts=None):
+    return _orig_rows(q, k, v, 1.0, key_counts)
 
 
-def _rows_scale_twice(q, k, v, scale):
-    return _orig_rows(q, k, v, scale * scale)
+def _rows_scale_twice(q, k, v, scale, key_counts=None):
+    return _orig_rows(q, k, v, scale * scale, key_counts)
 
 
-def _rows_transposed_v(q, k, v, scale):
-    o, l = _orig_rows(q, k, v, scale)
+def _rows_transposed_v(q, k, v, scale, key_counts=None):
+    o, l = _orig_rows(q, k, v, scale, key_counts)
     return o[:, ::-1].copy(), l                    # channel order reversed
 
 
-def _rows_drop_last_key(q, k, v, scale):
+def _rows_drop_last_key(q, k, v, scale, key_counts=None):
+    if key_counts is not None:
+        return _orig_rows(q, k, v, scale, key_counts)
     if k.shape[0] > 1:
         return _orig_rows(q, k[:-1], v[:-1], scale)
     return _orig_rows(q, k, v, scale)
+
+
+_orig_counts = O.causal_key_counts
+
+
+def _causal_counts_top_left(n_q, n_k):
+    return [min(i + 1, n_k) for i in range(n_q)]   # top-left instead of bottom-right alignment
+
+
+def _causal_counts_off_by_one(n_q, n_k):
+    return [max(c - 1, 0) for c in _orig_counts(n_q, n_k)]   # the diagonal key excluded
 
 
 def _merge_natural(o_parts, lse_parts):
@@ -58,6 +71,9 @@ PIN_TESTS = [
     lambda g: [P.test_merge_of_splits_equals_full(s) for s in range(4)],
     lambda g: P.test_merge_special_cases(),
     lambda g: P.test_chunked_merge_equals_full_with_smoothing(),
+    lambda g: P.test_causal_key_counts_hand_values(),
+    lambda g: [P.test_causal_against_torch_sdpa_float64(sq, sk) for sq, sk in [(7, 7), (5, 9), (9, 5)]],
+    lambda g: P.test_causal_decode_and_varlen_reduce_to_dense(),
 ]
 
 
@@ -78,6 +94,8 @@ def _some_pin_fails(golden_dir):
     ("last key dropped", "attention_rows", _rows_drop_last_key),
     ("merge weights in base e", "merge", _merge_natural),
     ("smoothing shift sign", "smooth_shift", _shift_wrong_sign),
+    ("causal mask aligned top-left", "causal_key_counts", _causal_counts_top_left),
+    ("causal mask misses the diagonal", "causal_key_counts", _causal_counts_off_by_one),
 ])
 def test_planted_mistake_is_caught(monkeypatch, golden_dir, name, attr, fn):
     monkeypatch.setattr(O, attr, fn)

@@ -453,3 +453,89 @@ def test_varlen_schedule_config4():
     order, offsets, items = O.varlen_schedule([0, 10, 10, 300, 310], [0, 5, 9, 9, 13], 2, 256)
     assert order == [0, 1, 3, 2]
     assert offsets == [0, 2, 2, 4, 8]
+
+
+# ------------------------------------------------------------ causal variant
+# (not on the pages; the reading: bottom-right alignment, see causal_key_counts)
+
+def test_causal_key_counts_hand_values():
+    assert O.causal_key_counts(4, 4) == [1, 2, 3, 4]
+    assert O.causal_key_counts(3, 5) == [3, 4, 5]       # 2 cached keys before the 3 queries
+    assert O.causal_key_counts(5, 3) == [0, 0, 1, 2, 3]  # the first 2 rows see nothing
+    assert O.causal_key_counts(1, 6) == [6]             # one decode row sees the whole cache
+    assert O.causal_key_counts(2, 0) == [0, 0]
+
+
+def _sdpa_masked(q, k, v, scale, allowed):
+    """PyTorch float64 reference with an explicit boolean mask (rows with no
+    allowed key excluded by the caller)."""
+    import torch
+    qt, kt, vt = (torch.from_numpy(np.ascontiguousarray(x)) for x in (q, k, v))
+    s = scale * qt @ kt.T
+    s = s.masked_fill(~torch.from_numpy(allowed), float("-inf"))
+    o = torch.nn.functional.scaled_dot_product_attention(qt[None, None], kt[None, None], vt[None, None],
+                                                         attn_mask=torch.from_numpy(allowed)[None, None],
+                                                         scale=scale)[0, 0]
+    return o.numpy(), (torch.logsumexp(s, dim=1) / math.log(2.0)).numpy()
+
+
+@pytest.mark.parametrize("sq,sk", [(7, 7), (5, 9), (9, 5), (1, 4), (16, 16)])
+def test_causal_against_torch_sdpa_float64(sq, sk):
+    rng = np.random.default_rng(sq * 31 + sk)
+    D = 8
+    q, k, v = rng.standard_normal((sq, D)) * 2, rng.standard_normal((sk, D)), rng.standard_normal((sk, D))
+    scale = D ** -0.5
+    i = np.arange(sq)[:, None]
+    j = np.arange(sk)[None, :]
+    allowed = j <= i + (sk - sq)                         # bottom-right aligned lower triangle
+    o, l = O.attention_rows(q, k, v, scale, O.causal_key_counts(sq, sk))
+    has = allowed.any(axis=1)
+    if has.any():
+        o_ref, l_ref = _sdpa_masked(q[has], k, v, scale, allowed[has])
+        np.testing.assert_allclose(o[has], o_ref, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(l[has], l_ref, rtol=1e-12, atol=1e-12)
+    assert np.all(o[~has] == 0) and np.all(np.isneginf(l[~has]))
+    if sq == sk:
+        import torch
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q)[None, None], torch.from_numpy(k)[None, None], torch.from_numpy(v)[None, None],
+            is_causal=True, scale=scale)[0, 0].numpy()
+        np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_causal_decode_and_varlen_reduce_to_dense():
+    import torch
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(2, 4, 3, 16, generator=g, dtype=torch.float64)
+    k = torch.randn(2, 2, 11, 16, generator=g, dtype=torch.float64)
+    v = torch.randn(2, 2, 11, 16, generator=g, dtype=torch.float64)
+    # decode rows are the last Lq positions of each kv_len-long sequence
+    o_d, l_d = O.decode(q, k, v, 0.25, kv_len=[11, 6], causal=True)
+    for b, n in enumerate([11, 6]):
+        o_ref, l_ref = O.dense(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n], 0.25, causal=True)
+        np.testing.assert_allclose(o_d[b:b + 1], o_ref, rtol=0, atol=0)
+        np.testing.assert_allclose(l_d[b:b + 1], l_ref, rtol=0, atol=0)
+    # one decode row sees every key: causal equals non-causal
+    o1, l1 = O.decode(q[:, :, :1], k, v, 0.25, causal=True)
+    o2, l2 = O.decode(q[:, :, :1], k, v, 0.25)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=0)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=0)
+    # row 0 of a 3-row causal decode over 11 keys sees exactly 9 of them
+    o9, l9 = O.attention_rows(O.to_f64(q[0, 0, :1]), O.to_f64(k[0, 0, :9]), O.to_f64(v[0, 0, :9]), 0.25)
+    np.testing.assert_allclose(o_d[0, 0, 0], o9[0], rtol=0, atol=0)
+    # varlen: each sequence is its own causal problem
+    lens_q, lens_k = [3, 0, 5], [4, 2, 5]
+    cq, ck = np.cumsum([0] + lens_q), np.cumsum([0] + lens_k)
+    qt = torch.randn(int(cq[-1]), 2, 8, generator=g, dtype=torch.float64)
+    kt = torch.randn(int(ck[-1]), 1, 8, generator=g, dtype=torch.float64)
+    vt = torch.randn(int(ck[-1]), 1, 8, generator=g, dtype=torch.float64)
+    o_v, l_v = O.varlen(qt, kt, vt, cq, ck, 0.5, causal=True)
+    for b in range(3):
+        if lens_q[b] == 0:
+            continue
+        qb = qt[cq[b]:cq[b + 1]].permute(1, 0, 2)[None]
+        kb = kt[ck[b]:ck[b + 1]].permute(1, 0, 2)[None]
+        vb = vt[ck[b]:ck[b + 1]].permute(1, 0, 2)[None]
+        o_ref, l_ref = O.dense(qb, kb, vb, 0.5, causal=True)
+        np.testing.assert_allclose(o_v[cq[b]:cq[b + 1]], o_ref[0].transpose(1, 0, 2), rtol=0, atol=0)
+        np.testing.assert_allclose(l_v[:, cq[b]:cq[b + 1]], l_ref[0], rtol=0, atol=0)
