@@ -126,6 +126,24 @@ skv_status attn_fwd_lse(const void* q, const void* k, const void* v, void* out, 
                         int max_seqlen_q, int max_seqlen_k, int smooth_k,
                         void* workspace, size_t workspace_bytes, skv_stream_t stream);
 
+/* attn_fwd_lse_causal: attn_fwd_lse with a causal mask.
+ *
+ * Not on the source pages (they use full, non-causal key ranges); the plainest
+ * adjacent variant, for autoregressive chunks: the len_q query rows of a
+ * sequence (batch entry or varlen sequence) are the LAST len_q positions of
+ * its len_k keys, so query row i sees keys j <= i + len_k - len_q
+ * (bottom-right alignment; the usual lower triangle when len_q == len_k).
+ * Rows i < len_q - len_k see no key: O = 0, LSE = -inf.  Arguments, layouts,
+ * workspace and errors as attn_fwd_lse; smooth_k subtracts the mean of the
+ * call's whole key range and still returns the unsmoothed LSE of the visible
+ * keys. */
+skv_status attn_fwd_lse_causal(const void* q, const void* k, const void* v, void* out, float* lse,
+                               int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                               skv_dtype dtype, skv_layout layout, const int32_t* cu_seqlens_q,
+                               const int32_t* cu_seqlens_k, int max_seqlen_q, int max_seqlen_k,
+                               int smooth_k, void* workspace, size_t workspace_bytes,
+                               skv_stream_t stream);
+
 /* Workspace bytes attn_fwd_lse needs for these arguments (0 if none).
  * Sk is the per-batch key length (dense) or total_k (TND). Host-only, pure. */
 size_t attn_fwd_lse_workspace(int B, int Hq, int Hkv, int Sk, int D, skv_dtype dtype,
@@ -162,6 +180,17 @@ skv_status attn_splitkv_decode(const void* q, const void* k, const void* v, void
                                float scale, skv_dtype dtype, const int32_t* kv_len,
                                int num_splits, void* workspace, size_t workspace_bytes,
                                skv_stream_t stream);
+
+/* attn_splitkv_decode_causal: attn_splitkv_decode with a causal mask over the
+ * Lq query rows (not on the source pages; the reading of attn_fwd_lse_causal):
+ * with n = kv_len[b] (or Lkv), query row i of [0, Lq) sees keys
+ * [0, n - Lq + 1 + i), so the last row sees the whole cache and Lq = 1 is the
+ * non-causal decode.  Arguments, workspace and errors as attn_splitkv_decode. */
+skv_status attn_splitkv_decode_causal(const void* q, const void* k, const void* v, void* out,
+                                      float* lse, int B, int Hq, int Hkv, int Lq, int Lkv, int D,
+                                      float scale, skv_dtype dtype, const int32_t* kv_len,
+                                      int num_splits, void* workspace, size_t workspace_bytes,
+                                      skv_stream_t stream);
 
 /* Split plan (host, pure integer).  For n keys, split s covers
  *   [s*C, min((s+1)*C, n)),  C = 64 * ceil(ceil(n / num_splits) / 64).

@@ -33,6 +33,8 @@ _c_int, _c_float, _c_size, _c_i64, _vp = ctypes.c_int, ctypes.c_float, ctypes.c_
 SIGNATURES = {
     "attn_fwd_lse": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                               _c_int, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
+    "attn_fwd_lse_causal": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                     _c_float, _c_int, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
     "attn_fwd_lse_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "attn_varlen_plan": (_c_int, [_vp, _vp, _c_int, _c_int, _vp, _vp]),
     "attn_splitkv_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -41,6 +43,8 @@ SIGNATURES = {
                                             _c_float, _c_int, _vp, _c_int, _vp]),
     "attn_splitkv_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp]),
     "attn_splitkv_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "attn_splitkv_decode_causal": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                            _c_float, _c_int, _vp, _c_int, _vp, _c_size, _vp]),
     "attn_splitkv_decode_fused": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                            _c_float, _c_int, _vp, _c_int, _vp, _c_size, _vp]),
     "attn_splitkv_workspace_init": (_c_int, [_vp, _c_size, _vp]),
@@ -183,7 +187,8 @@ def device_error() -> int:
 
 def attn_fwd_lse(q, k, v, scale: Optional[float] = None, layout: str = "HND", cu_seqlens_q=None,
                  cu_seqlens_k=None, max_seqlen_q: Optional[int] = None, max_seqlen_k: Optional[int] = None,
-                 smooth_k: int = 0, out=None, lse=None, return_lse: bool = True, workspace=None, stream=None):
+                 smooth_k: int = 0, out=None, lse=None, return_lse: bool = True, workspace=None, stream=None,
+                 causal: bool = False):
     """Attention forward with one log2 LSE per query row.
 
     Dense: q [B,Hq,Sq,D] (HND) or [B,Sq,Hq,D] (NHD), k/v likewise with Hkv, Sk.
@@ -192,6 +197,7 @@ def attn_fwd_lse(q, k, v, scale: Optional[float] = None, layout: str = "HND", cu
     (dense) or [Hq,total_q] (varlen), or (out, None) if return_lse is False.
     smooth_k: 0 off; 1 mean-shift applied to the fp32 logits; 2 K' = K - mean
     materialised in the input type.  Both return the LSE of the original logits.
+    causal: attn_fwd_lse_causal (query row i sees keys j <= i + len_k - len_q).
     """
     torch = _torch()
     _need_cuda(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k)
@@ -228,11 +234,11 @@ def attn_fwd_lse(q, k, v, scale: Optional[float] = None, layout: str = "HND", cu
     nbytes = attn_fwd_lse_workspace(B, Hq, Hkv, Sk, D, {0: "bf16", 1: "fp16", 2: "fp32"}[_dtype_code(q)],
                                     layout, smooth_k)
     workspace, wbytes = _workspace(nbytes, q.device, workspace)
-    st = lib().attn_fwd_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, float(scale),
-                            _dtype_code(q), LAYOUTS[layout], _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
-                            int(max_seqlen_q), int(max_seqlen_k), int(smooth_k), _ptr(workspace), wbytes,
-                            _stream(stream, q.device))
-    _check(st, "attn_fwd_lse")
+    fn = lib().attn_fwd_lse_causal if causal else lib().attn_fwd_lse
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, float(scale), _dtype_code(q),
+            LAYOUTS[layout], _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q), int(max_seqlen_k),
+            int(smooth_k), _ptr(workspace), wbytes, _stream(stream, q.device))
+    _check(st, "attn_fwd_lse_causal" if causal else "attn_fwd_lse")
     return out, lse
 
 
@@ -246,12 +252,15 @@ def attn_splitkv_workspace_init(workspace, stream=None):
 
 
 def attn_splitkv_decode(q, k, v, scale: Optional[float] = None, kv_len=None, num_splits: int = 0, out=None,
-                        lse=None, return_lse: bool = True, workspace=None, stream=None, fused: bool = False):
+                        lse=None, return_lse: bool = True, workspace=None, stream=None, fused: bool = False,
+                        causal: bool = False):
     """Split-KV decode: q [B,Hq,Lq,D], k/v [B,Hkv,Lkv,D] (HND).  kv_len: optional
     int32 device tensor [B].  num_splits 0 = automatic.  Returns (out, lse).
     fused=True: one kernel launch, the splits merged by the last CTA of each
     group (attn_splitkv_decode_fused); a workspace passed in must have been
-    zeroed once (attn_splitkv_workspace_init), one allocated here is zeroed."""
+    zeroed once (attn_splitkv_workspace_init), one allocated here is zeroed.
+    causal=True: attn_splitkv_decode_causal (row i of Lq sees the first
+    kv_len - Lq + 1 + i keys); not combined with fused."""
     torch = _torch()
     _need_cuda(q, k, v, out, lse, kv_len)
     B, Hq, Lq, D = q.shape
@@ -273,10 +282,14 @@ def attn_splitkv_decode(q, k, v, scale: Optional[float] = None, kv_len=None, num
     workspace, wbytes = _workspace(nbytes, q.device, workspace)
     if fused and fresh:
         attn_splitkv_workspace_init(workspace, stream)
-    fn = lib().attn_splitkv_decode_fused if fused else lib().attn_splitkv_decode
+    if fused and causal:
+        raise ValueError("the single-launch decode has no causal variant")
+    fn = lib().attn_splitkv_decode_fused if fused else (
+        lib().attn_splitkv_decode_causal if causal else lib().attn_splitkv_decode)
     st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lkv, D, float(scale), _dtype_code(q),
             _ptr(kv_len), int(splits), _ptr(workspace), wbytes, _stream(stream, q.device))
-    _check(st, "attn_splitkv_decode_fused" if fused else "attn_splitkv_decode")
+    _check(st, "attn_splitkv_decode_fused" if fused else (
+        "attn_splitkv_decode_causal" if causal else "attn_splitkv_decode"))
     return out, lse
 
 

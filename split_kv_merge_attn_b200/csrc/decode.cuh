@@ -62,6 +62,7 @@ struct DecodeArgs {
   int B, Hq, Hkv, Lq, Lkv;
   int num_splits;
   int row_groups;
+  int causal;  // 1: query row i (of Lq) sees keys j < kv_len - Lq + 1 + i
   float scale_log2;
 };
 
@@ -349,6 +350,16 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
       ldmatrix_x4(qs_addr + (r * Cfg::kQStride + c) * 2, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
     }
   }
+  // keys each of this thread's two tile rows (g, g + 8) may see: all of the
+  // split, or under the causal mask the first n - Lq + 1 + i keys of row i
+  int row_end[2] = {s1, s1};
+  if (a.causal) {
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int i = (rg * kDecodeRows + g + 8 * hr) % a.Lq;
+      row_end[hr] = min(s1, max(n - a.Lq + 1 + i, 0));
+    }
+  }
   float m[2] = {-INFINITY, -INFINITY};
   float lsum[2] = {0.f, 0.f};
   float o[D / 8][4];
@@ -393,7 +404,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int kidx = nt * 8 + 2 * tq + (e & 1);
-        const float val = (kidx < nvalid) ? sc[nt][e] * a.scale_log2 : -INFINITY;
+        const float val = (key0 + kidx < row_end[e >> 1]) ? sc[nt][e] * a.scale_log2 : -INFINITY;
         x[nt][e] = val;
       }
       mx0 = fmaxf(mx0, fmaxf(x[nt][0], x[nt][1]));

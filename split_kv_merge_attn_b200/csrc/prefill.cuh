@@ -133,6 +133,7 @@ struct PrefillArgs {
   int B, Hq, Hkv, Sq, Sk;
   int nqb;              // dense: 256-row query blocks per (b, h)
   int layout;           // 0 HND, 1 NHD, 2 TND
+  int causal;           // 1: row i of a sequence sees keys j <= i + len_k - len_q
   float scale_log2;
 };
 
@@ -197,7 +198,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int hkv = h / G;
   const int rows_here = min(2 * kPfBM, len_q - qblk * 2 * kPfBM);
   const int nt = rows_here > kPfBM ? 2 : 1;
-  const int nkv = (len_k + kPfBN - 1) / kPfBN;
+  // causal: rows are the last len_q positions of the key range (bottom-right
+  // alignment); the block stops at the KV tile holding its last row's last
+  // key, and both query tiles run over the same tiles (the first tile's rows
+  // simply see more masked keys)
+  const int causal_off = len_k - len_q;
+  const int kv_end = a.causal ? min(max(qblk * 2 * kPfBM + rows_here + causal_off, 0), len_k) : len_k;
+  const int nkv = (kv_end + kPfBN - 1) / kPfBN;
 
   // output addressing for query row qi (index inside the sequence)
   auto out_row = [&](int qi) -> T* {
@@ -395,6 +402,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint32_t o_addr = tmem + lane_base + (t == 0 ? Cfg::kOCol0 : Cfg::kOCol1);
       const int qi = qblk * 2 * kPfBM + t * kPfBM + row;  // row index inside the sequence
       const bool row_valid = qi < len_q;
+      const int row_keys = a.causal ? min(max(qi + causal_off + 1, 0), len_k) : len_k;  // keys this row sees
       bool ok = true;
 
       // smooth_k: delta = scale*log2(e) * (q_i . mean(K)), the shift smoothing removes
@@ -449,7 +457,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!ok) break;
         tc5::fence_after();
         // pass 1 over S (two halves of 64 columns read from TMEM): the row max
-        const int n_valid = len_k - j * kPfBN;
+        const int n_valid = row_keys - j * kPfBN;
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
@@ -501,7 +509,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // p = 2^(s * scale*log2(e) - max): P of keys [64h, 64h+64) is packed into
         // columns [32h, 32h+32) (logits this thread has already read) and
         // published on its own barrier, so PV can start on the first half
-        const float neg_bias = -(m_run + bias_shift);
+        // a row that has seen no key yet (causal rows before the first key)
+        // keeps m = -inf: exponentiate its masked logits against 0 instead
+        const float neg_bias = -((m_run == -INFINITY ? 0.f : m_run) + bias_shift);
         const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
         const uint64_t nb2 = f2_pack(neg_bias, neg_bias);
         uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -534,7 +544,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[t], 0, abort_flag, kErrPrefillWait));
       if (ok) {
         tc5::fence_after();
-        const float inv_l = 1.0f / l_run;
+        const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;  // no key: O = 0, LSE = -inf
         T* dst = row_valid ? out_row(qi) : nullptr;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {

@@ -180,11 +180,12 @@ size_t attn_fwd_lse_workspace(int B, int Hq, int Hkv, int Sk, int D, skv_dtype d
   return fwd_workspace(B, Hkv, Sk, D, layout, smooth_k).total;
 }
 
-skv_status attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+namespace {
+skv_status fwd_lse_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
                         int Sq, int Sk, int D, float scale, skv_dtype dtype, skv_layout layout,
                         const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int max_seqlen_q,
                         int max_seqlen_k, int smooth_k, void* workspace, size_t workspace_bytes,
-                        skv_stream_t stream) {
+                        skv_stream_t stream, int causal) {
   // ---- validation (no device work before it passes)
   if (q == nullptr || out == nullptr) return SKV_ERR_INVALID_ARG;
   if ((k == nullptr || v == nullptr) && Sk != 0) return SKV_ERR_INVALID_ARG;
@@ -232,6 +233,7 @@ skv_status attn_fwd_lse(const void* q, const void* k, const void* v, void* out, 
   p.scale = scale;
   p.dt = dtype;
   p.layout = layout;
+  p.causal = causal ? 1 : 0;
   if (varlen) {
     p.cu_q = cu_seqlens_q;
     p.cu_k = cu_seqlens_k;
@@ -259,13 +261,33 @@ skv_status attn_fwd_lse(const void* q, const void* k, const void* v, void* out, 
   }
   return cuda_status(skv::launch_prefill(p, stream));
 }
+}  // namespace
+
+skv_status attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                        int Sq, int Sk, int D, float scale, skv_dtype dtype, skv_layout layout,
+                        const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int max_seqlen_q,
+                        int max_seqlen_k, int smooth_k, void* workspace, size_t workspace_bytes,
+                        skv_stream_t stream) {
+  return fwd_lse_impl(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, dtype, layout, cu_seqlens_q, cu_seqlens_k,
+                      max_seqlen_q, max_seqlen_k, smooth_k, workspace, workspace_bytes, stream, 0);
+}
+
+skv_status attn_fwd_lse_causal(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                               int Hkv, int Sq, int Sk, int D, float scale, skv_dtype dtype, skv_layout layout,
+                               const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int max_seqlen_q,
+                               int max_seqlen_k, int smooth_k, void* workspace, size_t workspace_bytes,
+                               skv_stream_t stream) {
+  return fwd_lse_impl(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, dtype, layout, cu_seqlens_q, cu_seqlens_k,
+                      max_seqlen_q, max_seqlen_k, smooth_k, workspace, workspace_bytes, stream, 1);
+}
 
 // ------------------------------------------------------------------ decode
 
 namespace {
 skv_status decode_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
                        int Lq, int Lkv, int D, float scale, skv_dtype dtype, const int32_t* kv_len, int num_splits,
-                       void* workspace, size_t workspace_bytes, skv_stream_t stream, bool in_launch_merge) {
+                       void* workspace, size_t workspace_bytes, skv_stream_t stream, bool in_launch_merge,
+                       int causal) {
   if (q == nullptr || out == nullptr) return SKV_ERR_INVALID_ARG;
   if ((k == nullptr || v == nullptr) && Lkv != 0) return SKV_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return SKV_ERR_INVALID_ARG;
@@ -302,7 +324,7 @@ skv_status decode_impl(const void* q, const void* k, const void* v, void* out, f
     if (in_launch_merge) counters = reinterpret_cast<int*>(wsb + w.counters);
   }
   int e = skv::launch_decode(q, k, v, out, lse, part_o, part_lse, counters, kv_len, B, Hq, Hkv, Lq, Lkv, D, scale,
-                             dtype, splits, stream);
+                             dtype, splits, causal, stream);
   if (e) return cuda_status(e);
   if (splits > 1 && !in_launch_merge) {
     const int64_t rows = static_cast<int64_t>(B) * Hq * Lq;
@@ -319,7 +341,7 @@ skv_status attn_splitkv_decode(const void* q, const void* k, const void* v, void
                                int Hkv, int Lq, int Lkv, int D, float scale, skv_dtype dtype, const int32_t* kv_len,
                                int num_splits, void* workspace, size_t workspace_bytes, skv_stream_t stream) {
   return decode_impl(q, k, v, out, lse, B, Hq, Hkv, Lq, Lkv, D, scale, dtype, kv_len, num_splits, workspace,
-                     workspace_bytes, stream, /*in_launch_merge=*/false);
+                     workspace_bytes, stream, /*in_launch_merge=*/false, /*causal=*/0);
 }
 
 skv_status attn_splitkv_decode_fused(const void* q, const void* k, const void* v, void* out, float* lse, int B,
@@ -327,7 +349,15 @@ skv_status attn_splitkv_decode_fused(const void* q, const void* k, const void* v
                                      const int32_t* kv_len, int num_splits, void* workspace, size_t workspace_bytes,
                                      skv_stream_t stream) {
   return decode_impl(q, k, v, out, lse, B, Hq, Hkv, Lq, Lkv, D, scale, dtype, kv_len, num_splits, workspace,
-                     workspace_bytes, stream, /*in_launch_merge=*/true);
+                     workspace_bytes, stream, /*in_launch_merge=*/true, /*causal=*/0);
+}
+
+skv_status attn_splitkv_decode_causal(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                                      int Hq, int Hkv, int Lq, int Lkv, int D, float scale, skv_dtype dtype,
+                                      const int32_t* kv_len, int num_splits, void* workspace, size_t workspace_bytes,
+                                      skv_stream_t stream) {
+  return decode_impl(q, k, v, out, lse, B, Hq, Hkv, Lq, Lkv, D, scale, dtype, kv_len, num_splits, workspace,
+                     workspace_bytes, stream, /*in_launch_merge=*/false, /*causal=*/1);
 }
 
 skv_status attn_splitkv_workspace_init(void* workspace, size_t workspace_bytes, skv_stream_t stream) {

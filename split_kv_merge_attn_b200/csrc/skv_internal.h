@@ -47,7 +47,7 @@ int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, f
 // arrival counters, zero on entry, and the last CTA of each group merges.
 int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, float* part_o,
                   float* part_lse, int* counters, const int32_t* kv_len, int B, int Hq, int Hkv, int Lq, int Lkv,
-                  int D, float scale, skv_dtype dt, int num_splits, skv_stream_t stream);
+                  int D, float scale, skv_dtype dt, int num_splits, int causal, skv_stream_t stream);
 
 struct PrefillLaunch {
   const void* q;
@@ -58,6 +58,7 @@ struct PrefillLaunch {
   const float* kmean;      // [B(or seqs), Hkv, D] fp32 mean (materialised smooth_k), else null
   const float* kpartial;   // [chunks, B(or seqs), Hkv, D] per-256-key sums (shift smooth_k), else null
   int shift_logits;        // smooth_k == 1: apply the mean shift to the logits
+  int causal;              // bottom-right aligned causal mask
   const int32_t* cu_q;     // device, varlen only
   const int32_t* cu_k;
   const int32_t* order;    // device work order (varlen)

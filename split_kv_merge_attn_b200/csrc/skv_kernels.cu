@@ -190,7 +190,7 @@ int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeAr
 
 int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, float* part_o,
                   float* part_lse, int* counters, const int32_t* kv_len, int B, int Hq, int Hkv, int Lq, int Lkv,
-                  int D, float scale, skv_dtype dt, int num_splits, skv_stream_t stream) {
+                  int D, float scale, skv_dtype dt, int num_splits, int causal, skv_stream_t stream) {
   const int G = Hq / Hkv;
   DecodeArgs a;
   a.q = q;
@@ -206,6 +206,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
   a.Lq = Lq;
   a.Lkv = Lkv;
   a.num_splits = num_splits;
+  a.causal = causal;
   a.row_groups = static_cast<int>(ceil_div64(static_cast<int64_t>(G) * Lq, kDecodeRows));
   a.scale_log2 = scale * 1.4426950408889634f;
   // K and V as 2-D [B*Hkv*Lkv rows, D] maps; box = 64 columns x 64 keys
@@ -288,6 +289,7 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   a.kmean = p.kmean;
   a.kpartial = p.kpartial;
   a.shift_logits = p.shift_logits;
+  a.causal = p.causal;
   a.cu_q = p.cu_q;
   a.cu_k = p.cu_k;
   a.order = p.order;
