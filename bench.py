@@ -67,6 +67,9 @@ def decode_kv_bytes(Hkv, D, Lkv):
 
 
 MERGE5_BYTES = 4 * 16 * 4096 * (128 * 2 + 4) + 16 * 4096 * (128 * 2 + 4)
+# causal prefill of one workload-5 KV chunk (Sq = Sk = 4096, H = 16): the
+# visible (row, key) pairs are sum_i (i + 1)
+FLOPS_CAUSAL_CHUNK = attn_flops(16 * (4096 * 4097 // 2), D128)
 
 
 def load_peaks():
@@ -352,6 +355,20 @@ def run_ours(args, rank, world, dist):
     detail["merge_state_cfg5"] = {"graph_us": round(us_m, 2),
                                   "gbs": round(MERGE5_BYTES / (us_m * 1e-6) / 1e9, 1),
                                   "hbm_frac": round(MERGE5_BYTES / (us_m * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)}
+    # causal variants: prefill of the first workload-5 chunk with its own queries
+    # (Sq = Sk = 4096) and the Lq = 4 decode of workload 2 at Lkv 32768
+    oc = torch.empty_like(q5)
+    lc = torch.empty(1, 16, 4096, dtype=torch.float32, device=dev)
+    us_c = time_graph(lambda: skv.attn_fwd_lse(q5, k5[0], v5[0], scale, out=oc, lse=lc, causal=True), 20)
+    detail["causal_prefill_h16_s4096"] = {"graph_us": round(us_c, 2),
+                                          "tflops": round(FLOPS_CAUSAL_CHUNK / (us_c * 1e-6) / 1e12, 1)}
+    i4 = [n for n, *_r in DECODE_SHAPES].index("decode_d128_lq4_lkv32768")
+    _, qd, kd, vd, scd = dec_in[i4]
+    od, ld, wsd, spd = dec_buf[i4]
+    us_cd = time_graph(lambda: skv.attn_splitkv_decode(qd, kd, vd, scd, num_splits=spd, out=od, lse=ld, workspace=wsd,
+                                                       causal=True), 50)
+    detail["causal_decode_d128_lq4_lkv32768"] = {
+        "graph_us": round(us_cd, 2), "kv_gbs": round(decode_kv_bytes(8, 128, 32768) / (us_cd * 1e-6) / 1e9, 1)}
 
     # ---------------- end to end through the public API with host buffers
     e2e = run_e2e(args, dev, host, skv, torch, step_flops, world, dist)
