@@ -179,16 +179,32 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     len_q = a.cu_q[b + 1] - a.cu_q[b];
     len_k = a.cu_k[b + 1] - a.cu_k[b];
     const int nblk = (len_q + 2 * kPfBM - 1) / (2 * kPfBM);
-    h = rem / nblk;
-    qblk = rem % nblk;
+    if (a.causal) {
+      // causal work grows with the block index: the sequence's last (longest)
+      // blocks of every head start first
+      qblk = nblk - 1 - rem / a.Hq;
+      h = rem % a.Hq;
+    } else {
+      h = rem / nblk;
+      qblk = rem % nblk;
+    }
     q_row0 = a.cu_q[b] + qblk * 2 * kPfBM;
     k_row0 = a.cu_k[b];
     bcoord = 0;
   } else {
     const int item = blockIdx.x;
-    qblk = item % a.nqb;
-    h = (item / a.nqb) % a.Hq;
-    b = item / (a.nqb * a.Hq);
+    if (a.causal) {
+      // causal work grows with the block index: longest blocks (of every
+      // batch and head) first, so the grid runs longest-processing-time first
+      const int bh = item % (a.B * a.Hq);
+      qblk = a.nqb - 1 - item / (a.B * a.Hq);
+      h = bh % a.Hq;
+      b = bh / a.Hq;
+    } else {
+      qblk = item % a.nqb;
+      h = (item / a.nqb) % a.Hq;
+      b = item / (a.nqb * a.Hq);
+    }
     len_q = a.Sq;
     len_k = a.Sk;
     q_row0 = qblk * 2 * kPfBM;
