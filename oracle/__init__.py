@@ -38,7 +38,7 @@ __all__ = [
     "to_f64", "attention_rows", "dense", "varlen", "decode", "merge",
     "kv_mean", "smooth_shift", "smoothed_attention_rows", "chunked",
     "split_bounds", "auto_num_splits", "varlen_schedule", "lse_varlen_to_dense",
-    "causal_key_counts",
+    "causal_key_counts", "quantize_int8_blocks", "int8_attention_rows", "INT8_BLOCK",
 ]
 
 
@@ -258,6 +258,72 @@ def smoothed_attention_rows(q, k, v, scale: float, k_smoothed: Optional[np.ndarr
     kp = (k - mu[None]) if k_smoothed is None else np.asarray(k_smoothed, dtype=np.float64)
     o, lse_s = attention_rows(q, kp, v, scale)
     return o, lse_s + smooth_shift(q, mu, scale), lse_s
+
+
+# ---------------------------------------------------------------------------
+# INT8 QK^T with smooth_k (the variant smoothing exists for).
+# ---------------------------------------------------------------------------
+
+INT8_BLOCK = 128   # rows (query rows or keys) per quantization block
+
+
+def quantize_int8_blocks(x_rows, block: int = INT8_BLOCK) -> Tuple[np.ndarray, np.ndarray]:
+    """Symmetric int8 quantization with one scale per block of `block` rows.
+
+    ARK issue, Problem Description: smoothing K (subtracting its mean) is done
+    so that K quantizes well to INT8 in SageAttention-style kernels, with the
+    LSE of the original logits restored afterwards.  The pages give no
+    quantizer; the plainest reading, taken here: for the rows of one block,
+    amax = max |x| over the block, scale = amax / 127 (a block of zeros gets
+    scale 1), code = round-half-to-even(x / scale) clamped to [-127, 127].
+    All of it in fp32 (the values are fp32: 16-bit inputs widened, or K - mean
+    in fp32), so that the integer codes are decided in the kernel's precision.
+    Returns (codes int8 [n, D], scales fp32 [ceil(n / block)]).
+    """
+    x32 = np.asarray(x_rows, dtype=np.float32)
+    n = x32.shape[0]
+    nb = (n + block - 1) // block
+    codes = np.zeros(x32.shape, dtype=np.int8)
+    scales = np.ones(nb, dtype=np.float32)
+    for b in range(nb):
+        blk = x32[b * block:(b + 1) * block]
+        amax = np.float32(np.abs(blk).max()) if blk.size else np.float32(0.0)
+        sc = np.float32(amax / np.float32(127.0)) if amax > 0 else np.float32(1.0)
+        c = np.rint(blk / sc)                       # fp32 quotient, ties to even
+        codes[b * block:(b + 1) * block] = np.clip(c, -127, 127).astype(np.int8)
+        scales[b] = sc
+    return codes, scales
+
+
+def int8_attention_rows(q, k, v, scale: float, smooth: bool = True, mu: Optional[np.ndarray] = None,
+                        block: int = INT8_BLOCK) -> Tuple[np.ndarray, np.ndarray]:
+    """O and log2-LSE of query rows q [n, D] (one head) over keys k [m, D] with
+    Q K'^T taken from int8 codes.
+
+    K' = K - mean(K) over the call's keys (fp32; ``smooth=False`` quantizes K
+    itself), Q and K' quantized per block of rows (``quantize_int8_blocks``),
+    logits from the exact integer dot products,
+    s_ij = scale * sq_{block(i)} * sk_{block(j)} * (qc_i . kc_j), then the
+    plain definition (``attention_rows`` on those logits, via scaled codes) with
+    the 16-bit V, and the smoothing shift scale * (q_i . mean) / ln 2 added back
+    to the LSE (ARK issue, repro part 3).  ``mu`` may supply the fp32 mean.
+    """
+    q32 = np.asarray(q, dtype=np.float32)
+    k32 = np.asarray(k, dtype=np.float32)
+    n, m = q32.shape[0], k32.shape[0]
+    if m == 0:
+        return np.zeros((n, np.asarray(v).shape[1])), np.full(n, -np.inf)
+    if smooth:
+        mu32 = np.float32(kv_mean(k32)) if mu is None else np.asarray(mu, dtype=np.float32)
+    else:
+        mu32 = np.zeros(k32.shape[1], dtype=np.float32)
+    kp = (k32 - mu32[None]).astype(np.float32)
+    qc, qs = quantize_int8_blocks(q32, block)
+    kc, ks = quantize_int8_blocks(kp, block)
+    qd = qc.astype(np.float64) * np.repeat(qs.astype(np.float64), block)[:n, None]
+    kd = kc.astype(np.float64) * np.repeat(ks.astype(np.float64), block)[:m, None]
+    o, lse = attention_rows(qd, kd, v, scale)
+    return o, lse + smooth_shift(q32, mu32.astype(np.float64), scale)
 
 
 def chunked(q, k, v, scale: float, bounds: Sequence[int], layout: str = "HND"):

@@ -41,6 +41,21 @@ def _rows_drop_last_key(q, k, v, scale, key_counts=None):
 _orig_counts = O.causal_key_counts
 
 
+_orig_quant = O.quantize_int8_blocks
+
+
+def _quant_scale_128(x_rows, block=128):
+    codes, scales = _orig_quant(x_rows, block)
+    x32 = np.asarray(x_rows, dtype=np.float32)
+    out = codes.copy()
+    for b in range(len(scales)):
+        blk = x32[b * block:(b + 1) * block]
+        s = np.float32(np.abs(blk).max() / np.float32(128.0)) if blk.size and np.abs(blk).max() > 0 else np.float32(1)
+        out[b * block:(b + 1) * block] = np.clip(np.rint(blk / s), -127, 127).astype(np.int8)
+        scales[b] = s
+    return out, scales
+
+
 def _causal_counts_top_left(n_q, n_k):
     return [min(i + 1, n_k) for i in range(n_q)]   # top-left instead of bottom-right alignment
 
@@ -74,6 +89,9 @@ PIN_TESTS = [
     lambda g: P.test_causal_key_counts_hand_values(),
     lambda g: [P.test_causal_against_torch_sdpa_float64(sq, sk) for sq, sk in [(7, 7), (5, 9), (9, 5)]],
     lambda g: P.test_causal_decode_and_varlen_reduce_to_dense(),
+    lambda g: P.test_int8_quantizer_properties(),
+    lambda g: P.test_int8_attention_is_exact_for_representable_inputs(),
+    lambda g: P.test_int8_smoothing_is_what_makes_int8_keys_accurate(),
 ]
 
 
@@ -96,6 +114,7 @@ def _some_pin_fails(golden_dir):
     ("smoothing shift sign", "smooth_shift", _shift_wrong_sign),
     ("causal mask aligned top-left", "causal_key_counts", _causal_counts_top_left),
     ("causal mask misses the diagonal", "causal_key_counts", _causal_counts_off_by_one),
+    ("int8 scale amax / 128", "quantize_int8_blocks", _quant_scale_128),
 ])
 def test_planted_mistake_is_caught(monkeypatch, golden_dir, name, attr, fn):
     monkeypatch.setattr(O, attr, fn)

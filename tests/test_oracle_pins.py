@@ -539,3 +539,64 @@ def test_causal_decode_and_varlen_reduce_to_dense():
         o_ref, l_ref = O.dense(qb, kb, vb, 0.5, causal=True)
         np.testing.assert_allclose(o_v[cq[b]:cq[b + 1]], o_ref[0].transpose(1, 0, 2), rtol=0, atol=0)
         np.testing.assert_allclose(l_v[:, cq[b]:cq[b + 1]], l_ref[0], rtol=0, atol=0)
+
+
+# ------------------------------------------------------------ INT8 QK^T with smooth_k
+
+def test_int8_quantizer_properties():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((300, 16)) * rng.uniform(0.1, 9.0, (300, 1))).astype(np.float32)
+    x[128:256] = 0.0                                   # an all-zero block
+    codes, scales = O.quantize_int8_blocks(x, 128)
+    assert codes.dtype == np.int8 and scales.shape == (3,)
+    assert np.all(np.abs(codes.astype(int)) <= 127)
+    assert scales[1] == 1.0 and np.all(codes[128:256] == 0)
+    for b in (0, 2):
+        blk = x[b * 128:(b + 1) * 128]
+        s = np.float32(np.abs(blk).max() / np.float32(127))
+        assert scales[b] == s
+        i = np.unravel_index(np.abs(blk).argmax(), blk.shape)
+        assert abs(int(codes[b * 128:][i])) == 127                 # the block's largest value maps to +-127
+        err = np.abs(blk.astype(np.float64) - codes[b * 128:(b + 1) * 128].astype(np.float64) * s)
+        assert err.max() <= 0.5 * s * (1 + 1e-5)                    # round to nearest
+    # ties go to even: x / s = 2.5 -> 2, 3.5 -> 4, -0.5 -> 0
+    t = np.array([[2.5, 3.5, -0.5, 127.0]], dtype=np.float32)
+    c, s = O.quantize_int8_blocks(t, 128)
+    assert s[0] == 1.0 and c.tolist() == [[2, 4, 0, 127]]
+
+
+def test_int8_attention_is_exact_for_representable_inputs():
+    """Inputs whose codes lose nothing (integer multiples of a power of two,
+    each block reaching +-127, keys with exactly zero mean) reduce to the plain
+    definition."""
+    rng = np.random.default_rng(4)
+    D = 16
+    qc = rng.integers(-127, 128, (40, D))
+    qc[0, 0] = 127                                     # one query block, reaching 127
+    half = rng.integers(-127, 128, (100, D))
+    half[0, 0] = 127                                   # block 0 (keys 0..127) reaches 127
+    half[50, 0] = 127                                  # key 150 = -127 lies in block 1
+    kc = np.concatenate([half, -half])                 # every channel sums to zero
+    q = (qc * 2.0 ** -5).astype(np.float32)
+    k = (kc * 2.0 ** -6).astype(np.float32)
+    assert np.all(k.astype(np.float64).sum(axis=0) == 0)
+    v = rng.standard_normal((200, D))
+    o8, l8 = O.int8_attention_rows(q, k, v, 0.3)
+    o, l = O.attention_rows(q, k, v, 0.3)
+    np.testing.assert_allclose(o8, o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(l8, l, rtol=1e-12, atol=1e-12)
+
+
+def test_int8_smoothing_is_what_makes_int8_keys_accurate():
+    """The reason smooth_k exists (ARK issue): with a per-channel offset in K,
+    quantizing K' = K - mean loses far less than quantizing K."""
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((64, 32)) * 2
+    k = rng.standard_normal((512, 32)) + 6.0
+    v = rng.standard_normal((512, 32))
+    o, l = O.attention_rows(q, k, v, 32 ** -0.5)
+    o_s, l_s = O.int8_attention_rows(q, k, v, 32 ** -0.5, smooth=True)
+    o_n, l_n = O.int8_attention_rows(q, k, v, 32 ** -0.5, smooth=False)
+    e_s, e_n = np.abs(l_s - l).max(), np.abs(l_n - l).max()
+    assert e_s < 0.05 and e_n > 5 * e_s
+    assert np.abs(o_s - o).max() < np.abs(o_n - o).max()
