@@ -144,6 +144,32 @@ skv_status attn_fwd_lse_causal(const void* q, const void* k, const void* v, void
                                int smooth_k, void* workspace, size_t workspace_bytes,
                                skv_stream_t stream);
 
+/* attn_fwd_lse_int8: attention with Q K'^T computed from INT8 codes.
+ *
+ * ARK issue, Problem Description: K is smoothed (its mean over the call's keys
+ * subtracted) so that it quantizes well to INT8, and the LSE of the original
+ * logits is restored with the q . mean(K) shift.  Here: K' = K - mean (fp32)
+ * and Q are quantized per block of 128 rows (symmetric, scale = amax / 127,
+ * round half to even), S is the exact s32 product of the codes on the int8
+ * tensor cores times the two block scales, and the softmax and P V (V in
+ * 16-bit) are those of attn_fwd_lse; LSE = log2 sum_j exp(s_ij) + the shift.
+ * Results approximate attn_fwd_lse to the quantization error (logits to about
+ * 1e-2 for randn-like inputs); they are exact for inputs the codes represent.
+ * Dense HND only: q [B,Hq,Sq,128], k/v [B,Hkv,Sk,128], out like q, lse
+ * [B,Hq,Sq] fp32 (nullable); bf16 or fp16; causal 0/1 as attn_fwd_lse_causal.
+ * workspace (device, 256-byte aligned, >= attn_fwd_lse_int8_workspace bytes)
+ * holds, each section 256-byte aligned and in this order: fp32 column sums
+ * [ceil(Sk/256), B, Hkv, 128], fp32 mean [B, Hkv, 128], Q codes int8
+ * [B, Hq, Sq, 128], K' codes int8 [B, Hkv, Sk, 128], fp32 Q block scales
+ * [B, Hq, ceil(Sq/128)], fp32 K' block scales [B, Hkv, ceil(Sk/128)], fp32
+ * shift [B, Hq, Sq].  Errors as attn_fwd_lse; SKV_ERR_UNSUPPORTED for D != 128,
+ * fp32, or B*Hq > 65535. */
+skv_status attn_fwd_lse_int8(const void* q, const void* k, const void* v, void* out, float* lse,
+                             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                             skv_dtype dtype, int causal, void* workspace, size_t workspace_bytes,
+                             skv_stream_t stream);
+size_t attn_fwd_lse_int8_workspace(int B, int Hq, int Hkv, int Sq, int Sk, int D);
+
 /* Workspace bytes attn_fwd_lse needs for these arguments (0 if none).
  * Sk is the per-batch key length (dense) or total_k (TND). Host-only, pure. */
 size_t attn_fwd_lse_workspace(int B, int Hq, int Hkv, int Sk, int D, skv_dtype dtype,

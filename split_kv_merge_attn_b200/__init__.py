@@ -35,6 +35,9 @@ SIGNATURES = {
                               _c_int, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
     "attn_fwd_lse_causal": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_float, _c_int, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
+    "attn_fwd_lse_int8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                                   _c_int, _c_int, _vp, _c_size, _vp]),
+    "attn_fwd_lse_int8_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "attn_fwd_lse_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "attn_varlen_plan": (_c_int, [_vp, _vp, _c_int, _c_int, _vp, _vp]),
     "attn_splitkv_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -239,6 +242,34 @@ def attn_fwd_lse(q, k, v, scale: Optional[float] = None, layout: str = "HND", cu
             LAYOUTS[layout], _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q), int(max_seqlen_k),
             int(smooth_k), _ptr(workspace), wbytes, _stream(stream, q.device))
     _check(st, "attn_fwd_lse_causal" if causal else "attn_fwd_lse")
+    return out, lse
+
+
+def attn_fwd_lse_int8_workspace(B: int, Hq: int, Hkv: int, Sq: int, Sk: int, D: int = 128) -> int:
+    return int(lib().attn_fwd_lse_int8_workspace(B, Hq, Hkv, Sq, Sk, D))
+
+
+def attn_fwd_lse_int8(q, k, v, scale: Optional[float] = None, causal: bool = False, out=None, lse=None,
+                      return_lse: bool = True, workspace=None, stream=None):
+    """Attention with Q K'^T from INT8 codes of Q and of the smoothed K
+    (dense HND, D = 128).  Returns (out, lse [B,Hq,Sq])."""
+    torch = _torch()
+    _need_cuda(q, k, v, out, lse)
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Sk, _ = k.shape
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if not return_lse:
+        lse = None
+    workspace, wbytes = _workspace(attn_fwd_lse_int8_workspace(B, Hq, Hkv, Sq, Sk, D), q.device, workspace)
+    st = lib().attn_fwd_lse_int8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D,
+                                 float(scale), _dtype_code(q), int(bool(causal)), _ptr(workspace), wbytes,
+                                 _stream(stream, q.device))
+    _check(st, "attn_fwd_lse_int8")
     return out, lse
 
 

@@ -99,12 +99,32 @@ __device__ __forceinline__ void exp_pack_64(const float (&sv)[64], uint64_t sc2,
   }
 }
 
-template <int D>
+// kI8: Q and K arrive as int8 codes (one 128-byte box per row at D = 128)
+// and S = Q K^T is an s32 .kind::i8 product; V stays 16-bit.
+// s32 logits read from TMEM (bit patterns in float registers) to exact fp32
+// values: |s| < 2^22 for int8 codes at D <= 128, so adding the bits of
+// 1.5 * 2^23 and subtracting it again is exact.
+__device__ __forceinline__ void s32_to_f32_64(float (&v)[64]) {
+  const uint64_t neg_magic = f2_pack(-12582912.0f, -12582912.0f);
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    const float a0 = __int_as_float(__float_as_int(v[c]) + 0x4B400000);
+    const float a1 = __int_as_float(__float_as_int(v[c + 1]) + 0x4B400000);
+    const float2 r = f2_unpack(fadd2(f2_pack(a0, a1), neg_magic));
+    v[c] = r.x;
+    v[c + 1] = r.y;
+  }
+}
+
+template <int D, bool kI8 = false>
 struct PrefillCfg {
-  static constexpr int kBoxes = D / 64;
+  static constexpr int kBoxes = D / 64;              // 64-element boxes of a 16-bit row (V, and Q/K)
+  static constexpr int kQKBoxes = kI8 ? D / 128 : kBoxes;  // boxes of a Q or K row
+  static constexpr int kQKBoxElems = kI8 ? 128 : 64;
   static constexpr int kBoxBytes = 128 * 128;       // 128 rows x 128 bytes
-  static constexpr int kQTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kKVTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kQTileBytes = kQKBoxes * kBoxBytes;
+  static constexpr int kKTileBytes = kQKBoxes * kBoxBytes;
+  static constexpr int kKVTileBytes = kBoxes * kBoxBytes;   // one ring buffer (a V tile; a K tile fits)
   static constexpr int kStages = (D == 64) ? 8 : 5;
   static constexpr int kRingBytes = kStages * kKVTileBytes;
   static constexpr int kOffQ = 0;
@@ -122,6 +142,9 @@ struct PrefillCfg {
 struct PrefillArgs {
   void* out;
   float* lse;
+  const float* qscale;  // int8: [B, Hq, ceil(Sq/128)] scale of each 128-row block of Q codes
+  const float* kscale;  // int8: [B, Hkv, ceil(Sk/128)] scale of each 128-key block of K' codes
+  const float* dq;      // int8: [B, Hq, Sq] smoothing shift scale*log2(e)*(q . mean K), added to the LSE
   const float* kmean;   // smooth (materialised K'): [Bseq, Hkv, D] fp32 mean, else null
   const float* kpartial;  // smooth (logit shift): [chunks, Bseq, Hkv, D] per-256-key column sums, else null
   int shift_logits;     // smooth: 1 = subtract the mean term from the fp32 logits (K unsmoothed),
@@ -137,13 +160,14 @@ struct PrefillArgs {
   float scale_log2;
 };
 
-template <int D, typename T>
+template <int D, typename T, bool kI8 = false>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
-  using Cfg = PrefillCfg<D>;
+  using Cfg = PrefillCfg<D, kI8>;
+  static_assert(!kI8 || D == 128, "the int8 path has one 128-byte box per row");
   constexpr int kIsBf16 = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
-  constexpr uint32_t kIdescQK = tc5::idesc_f16(kIsBf16, 0, kPfBM, kPfBN);
+  constexpr uint32_t kIdescQK = kI8 ? tc5::idesc_i8(kPfBM, kPfBN) : tc5::idesc_f16(kIsBf16, 0, kPfBM, kPfBN);
   constexpr uint32_t kIdescPV = tc5::idesc_f16(kIsBf16, 1, kPfBM, D);
 
   extern __shared__ uint8_t smem_raw[];
@@ -279,9 +303,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int t = 0; t < nt; ++t) {
         const int s = q_row0 + t * kPfBM;
 #pragma unroll
-        for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-          if (hnd) tma_load_4d(qtile[t] + bx * Cfg::kBoxBytes, &tmQ, q_full, bx * 64, s, h, bcoord);
-          else tma_load_4d(qtile[t] + bx * Cfg::kBoxBytes, &tmQ, q_full, bx * 64, h, s, bcoord);
+        for (int bx = 0; bx < Cfg::kQKBoxes; ++bx) {
+          const int x = bx * Cfg::kQKBoxElems;
+          if (hnd) tma_load_4d(qtile[t] + bx * Cfg::kBoxBytes, &tmQ, q_full, x, s, h, bcoord);
+          else tma_load_4d(qtile[t] + bx * Cfg::kBoxBytes, &tmQ, q_full, x, h, s, bcoord);
         }
       }
       int issued = 0;
@@ -297,13 +322,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               break;
             }
           }
-          mbar_arrive_expect_tx(&kv_full[buf], Cfg::kKVTileBytes);
           const CUtensorMap* m = which ? &tmV : &tmK;
+          const int nbox = which ? Cfg::kBoxes : Cfg::kQKBoxes;
+          const int bxe = which ? 64 : Cfg::kQKBoxElems;
+          mbar_arrive_expect_tx(&kv_full[buf], which ? Cfg::kKVTileBytes : Cfg::kKTileBytes);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+            if (bx >= nbox) break;
             uint8_t* dst = ring + buf * Cfg::kKVTileBytes + bx * Cfg::kBoxBytes;
-            if (hnd) tma_load_4d(dst, m, &kv_full[buf], bx * 64, s, hkv, bcoord);
-            else tma_load_4d(dst, m, &kv_full[buf], bx * 64, hkv, s, bcoord);
+            if (hnd) tma_load_4d(dst, m, &kv_full[buf], bx * bxe, s, hkv, bcoord);
+            else tma_load_4d(dst, m, &kv_full[buf], bx * bxe, hkv, s, bcoord);
           }
           issued = u + 1;
         }
@@ -336,10 +364,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint64_t dv_base = tc5::smem_desc(ring_addr, Cfg::kBoxBytes, 1024);
       auto issue_s = [&](uint64_t dq, uint32_t sc, int u) {
         const uint64_t dk = dk_base + static_cast<uint64_t>(((u % Cfg::kStages) * Cfg::kKVTileBytes) >> 4);
+        // one MMA per 32 bytes of a Q/K row (K = 16 for 16-bit, 32 for int8)
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < (kI8 ? D / 32 : D / 16); ++kk) {
           const uint64_t o = static_cast<uint64_t>(((kk >> 2) * Cfg::kBoxBytes + (kk & 3) * 32) >> 4);
-          tc5::mma_ss(sc, dq + o, dk + o, kIdescQK, kk > 0 ? 1u : 0u);
+          if constexpr (kI8) tc5::mma_ss_i8(sc, dq + o, dk + o, kIdescQK, kk > 0 ? 1u : 0u);
+          else tc5::mma_ss(sc, dq + o, dk + o, kIdescQK, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv_half = [&](uint32_t sc, uint32_t oc, int u, bool acc, int hf) {
@@ -466,12 +496,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // logits seen by the softmax are the smoothed ones: K' = K - mean either
       // materialised (K' in the MMA) or applied here as a per-row fp32 shift
       const float bias_shift = a.shift_logits ? delta : 0.f;
+      // int8: a logit is s32 codes-product x (Q block scale x K block scale);
+      // the K scale of the next KV tile is fetched one tile ahead
+      float qsc = 1.f, ks_next = 1.f;
+      const float* ksc = nullptr;
+      if constexpr (kI8) {
+        qsc = __ldg(a.qscale + (static_cast<int64_t>(b) * a.Hq + h) * ((a.Sq + 127) / 128) + qblk * 2 + t);
+        ksc = a.kscale + (static_cast<int64_t>(b) * a.Hkv + hkv) * ((a.Sk + 127) / 128);
+        ks_next = __ldg(ksc);
+        if (row_valid) delta = __ldg(a.dq + (static_cast<int64_t>(b) * a.Hq + h) * a.Sq + qi);
+      }
       float m_run = -INFINITY;  // running max of the (smoothed) log2-domain logits, possibly stale
       float l_run = 0.f;
       for (int j = 0; j < nkv && ok; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, kErrPrefillWait));
         if (!ok) break;
         tc5::fence_after();
+        float sl2 = a.scale_log2;  // log2 units per logit unit of this tile
+        if constexpr (kI8) {
+          sl2 = a.scale_log2 * qsc * ks_next;
+          if (j + 1 < nkv) ks_next = __ldg(ksc + j + 1);
+        }
         // pass 1 over S (two halves of 64 columns read from TMEM): the row max
         const int n_valid = row_keys - j * kPfBN;
         float mx8[8];
@@ -483,6 +528,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tc5::ld32(s_addr + hf * 64, *reinterpret_cast<float(*)[32]>(&sh[0]));
           tc5::ld32(s_addr + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
           tc5::wait_ld();
+          if constexpr (kI8) s32_to_f32_64(sh);
           if (n_valid < kPfBN) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
@@ -494,7 +540,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], sh[c + e], sh[c + 8 + e]);
         }
         const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-        const float t_max = fmaf(mx, a.scale_log2, -bias_shift);
+        const float t_max = fmaf(mx, sl2, -bias_shift);
         const float m_new = fmaxf(m_run, t_max);
         const bool rescale = m_new > m_run + kPfRescaleThreshold;
         float alpha = 1.f;
@@ -528,7 +574,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // a row that has seen no key yet (causal rows before the first key)
         // keeps m = -inf: exponentiate its masked logits against 0 instead
         const float neg_bias = -((m_run == -INFINITY ? 0.f : m_run) + bias_shift);
-        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
+        const uint64_t sc2 = f2_pack(sl2, sl2);
         const uint64_t nb2 = f2_pack(neg_bias, neg_bias);
         uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
         const bool full_tile = n_valid >= kPfBN;  // masked tails stay on the MUFU (exact zeros)
@@ -538,6 +584,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tc5::ld32(s_addr + hf * 64, *reinterpret_cast<float(*)[32]>(&sh[0]));
           tc5::ld32(s_addr + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
           tc5::wait_ld();
+          if constexpr (kI8) s32_to_f32_64(sh);
           if (!full_tile) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)

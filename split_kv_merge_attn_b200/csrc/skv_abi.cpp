@@ -281,6 +281,88 @@ skv_status attn_fwd_lse_causal(const void* q, const void* k, const void* v, void
                       max_seqlen_q, max_seqlen_k, smooth_k, workspace, workspace_bytes, stream, 1);
 }
 
+// ------------------------------------------------------------------ int8 prefill
+
+namespace {
+struct Int8Ws {
+  size_t partial = 0, kmean = 0, q8 = 0, k8 = 0, qs = 0, ks = 0, dq = 0, total = 0;
+};
+Int8Ws int8_ws_layout(int B, int Hq, int Hkv, int Sq, int Sk) {
+  Int8Ws w;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += skv::align256(bytes);
+    return o;
+  };
+  const size_t b = static_cast<size_t>(B);
+  w.partial = take(static_cast<size_t>((Sk + 255) / 256) * b * Hkv * 128 * 4);
+  w.kmean = take(b * Hkv * 128 * 4);
+  w.q8 = take(b * Hq * static_cast<size_t>(Sq) * 128);
+  w.k8 = take(b * Hkv * static_cast<size_t>(Sk) * 128);
+  w.qs = take(b * Hq * static_cast<size_t>((Sq + 127) / 128) * 4);
+  w.ks = take(b * Hkv * static_cast<size_t>((Sk + 127) / 128) * 4);
+  w.dq = take(b * Hq * static_cast<size_t>(Sq) * 4);
+  w.total = off;
+  return w;
+}
+}  // namespace
+
+size_t attn_fwd_lse_int8_workspace(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 0 || Sk < 0 || D != 128) return 0;
+  return int8_ws_layout(B, Hq, Hkv, Sq, Sk).total;
+}
+
+skv_status attn_fwd_lse_int8(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                             int Hkv, int Sq, int Sk, int D, float scale, skv_dtype dtype, int causal,
+                             void* workspace, size_t workspace_bytes, skv_stream_t stream) {
+  if (q == nullptr || out == nullptr) return SKV_ERR_INVALID_ARG;
+  if ((k == nullptr || v == nullptr) && Sk != 0) return SKV_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return SKV_ERR_INVALID_ARG;
+  if (lse != nullptr && !aligned(lse, 4)) return SKV_ERR_INVALID_ARG;
+  if (dtype != SKV_BF16 && dtype != SKV_FP16 && dtype != SKV_FP32) return SKV_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || D < 1 || Sq < 0 || Sk < 0 || Hq % Hkv != 0) return SKV_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SKV_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SKV_ERR_INVALID_ARG;
+  if (!is_half_type(dtype) || D != 128) return SKV_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * Hq > 65535) return SKV_ERR_UNSUPPORTED;  // grid.y of the code kernels
+  if (static_cast<int64_t>(B) * Hq * skv::ceil_div64(Sq, skv::kPrefillRowsPerCta) > 0x7fffffff)
+    return SKV_ERR_UNSUPPORTED;
+  if (Sq == 0) return SKV_OK;
+  if (Sk == 0) {  // no keys: O = 0, LSE = -inf, as the 16-bit path writes them
+    return causal ? attn_fwd_lse_causal(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, dtype, SKV_HND, nullptr,
+                                        nullptr, 0, 0, 0, nullptr, 0, stream)
+                  : attn_fwd_lse(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, dtype, SKV_HND, nullptr, nullptr,
+                                 0, 0, 0, nullptr, 0, stream);
+  }
+  const Int8Ws w = int8_ws_layout(B, Hq, Hkv, Sq, Sk);
+  if (workspace_bytes < w.total) return SKV_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace == nullptr || !aligned(workspace, 256)) return SKV_ERR_INVALID_ARG;
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  skv::Int8PrefillLaunch p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.out = out;
+  p.lse = lse;
+  p.kpartial = reinterpret_cast<float*>(wsb + w.partial);
+  p.kmean = reinterpret_cast<float*>(wsb + w.kmean);
+  p.q8 = reinterpret_cast<int8_t*>(wsb + w.q8);
+  p.k8 = reinterpret_cast<int8_t*>(wsb + w.k8);
+  p.qscale = reinterpret_cast<float*>(wsb + w.qs);
+  p.kscale = reinterpret_cast<float*>(wsb + w.ks);
+  p.dq = reinterpret_cast<float*>(wsb + w.dq);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.scale = scale;
+  p.dt = dtype;
+  p.causal = causal;
+  return cuda_status(skv::launch_prefill_int8(p, stream));
+}
+
 // ------------------------------------------------------------------ decode
 
 namespace {

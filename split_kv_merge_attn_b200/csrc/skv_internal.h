@@ -71,6 +71,29 @@ struct PrefillLaunch {
 };
 int launch_prefill(const PrefillLaunch& p, skv_stream_t stream);
 
+// INT8 Q K'^T prefill (dense HND, D = 128): mean of K, int8 codes of K - mean
+// and of Q with their per-128-row scales and the per-row smoothing shift, then
+// the prefill over the codes.  All buffers device, caller-owned.
+struct Int8PrefillLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;
+  float* kpartial;  // [ceil(Sk/256), B, Hkv, 128]
+  float* kmean;     // [B, Hkv, 128]
+  int8_t* q8;       // [B, Hq, Sq, 128]
+  int8_t* k8;       // [B, Hkv, Sk, 128]
+  float* qscale;    // [B, Hq, ceil(Sq/128)]
+  float* kscale;    // [B, Hkv, ceil(Sk/128)]
+  float* dq;        // [B, Hq, Sq]
+  int B, Hq, Hkv, Sq, Sk;
+  float scale;
+  skv_dtype dt;
+  int causal;
+};
+int launch_prefill_int8(const Int8PrefillLaunch& p, skv_stream_t stream);
+
 int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int32_t* order,
                        int32_t* offsets, skv_stream_t stream);
 

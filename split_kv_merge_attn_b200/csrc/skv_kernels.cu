@@ -13,6 +13,7 @@
 #include "skv_device.cuh"
 #include "merge_state.cuh"
 #include "decode.cuh"
+#include "quant.cuh"
 #include "prefill.cuh"
 #include "smooth.cuh"
 
@@ -72,8 +73,8 @@ CUtensorMapDataType tmap_type(skv_dtype dt) {
 
 // Tiled map over a 16-bit tensor of `rank` dims (dims[0] innermost, strides in
 // bytes for dims 1..rank-1), box {64, box1, ...}, 128-byte swizzle, zero fill.
-int make_tmap(CUtensorMap* m, skv_dtype dt, int rank, const void* base, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box) {
+int make_tmap_ty(CUtensorMap* m, CUtensorMapDataType ty, int rank, const void* base, const uint64_t* dims,
+                 const uint64_t* strides_bytes, const uint32_t* box) {
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   int e = get_encoder(&enc);
   if (e) return e;
@@ -86,10 +87,15 @@ int make_tmap(CUtensorMap* m, skv_dtype dt, int rank, const void* base, const ui
     es[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) gstr[i] = strides_bytes[i];
-  CUresult r = enc(m, tmap_type(dt), static_cast<cuuint32_t>(rank), const_cast<void*>(base), gdim, gstr, bx, es,
+  CUresult r = enc(m, ty, static_cast<cuuint32_t>(rank), const_cast<void*>(base), gdim, gstr, bx, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : static_cast<int>(cudaErrorInvalidValue);
+}
+
+int make_tmap(CUtensorMap* m, skv_dtype dt, int rank, const void* base, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_tmap_ty(m, tmap_type(dt), rank, base, dims, strides_bytes, box);
 }
 }  // namespace
 
@@ -257,11 +263,20 @@ int make_qkv_map(CUtensorMap* m, const void* base, skv_dtype dt, skv_layout layo
   return make_tmap(m, dt, 4, base, dims, strides, box);
 }
 
-template <int D, typename T>
+// int8 codes [B, H, S, 128] (HND) as a 4-D map (D, S, H, B), box 128 x 128 rows
+int make_i8_map(CUtensorMap* m, const void* base, int B, int H, int S) {
+  const uint64_t D = 128;
+  const uint64_t dims[4] = {D, static_cast<uint64_t>(S), static_cast<uint64_t>(H), static_cast<uint64_t>(B)};
+  const uint64_t strides[3] = {D, static_cast<uint64_t>(S) * D, static_cast<uint64_t>(H) * S * D};
+  const uint32_t box[4] = {128, 128, 1, 1};
+  return make_tmap_ty(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box);
+}
+
+template <int D, typename T, bool kI8 = false>
 int launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillArgs& a,
                      unsigned grid, cudaStream_t st) {
-  using Cfg = PrefillCfg<D>;
-  auto kern = prefill_kernel<D, T>;
+  using Cfg = PrefillCfg<D, kI8>;
+  auto kern = prefill_kernel<D, T, kI8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kPfThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, a);
@@ -286,6 +301,9 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   PrefillArgs a;
   a.out = p.out;
   a.lse = p.lse;
+  a.qscale = nullptr;
+  a.kscale = nullptr;
+  a.dq = nullptr;
   a.kmean = p.kmean;
   a.kpartial = p.kpartial;
   a.shift_logits = p.shift_logits;
@@ -321,6 +339,90 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
     if (p.D == 128) return launch_prefill_t<128, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
   }
   return cudaErrorInvalidValue;
+}
+
+int launch_prefill_int8(const Int8PrefillLaunch& p, skv_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int nqb = static_cast<int>(ceil_div64(p.Sq, kQuantBlock));
+  const int nkb = static_cast<int>(ceil_div64(p.Sk, kQuantBlock));
+  int launches = 0;
+  // fp32 mean of K over the call's keys: per-256-key column sums, then the mean
+  SmoothArgs sa;
+  sa.k = p.k;
+  sa.k_out = nullptr;
+  sa.partial = p.kpartial;
+  sa.kmean = p.kmean;
+  sa.cu_k = nullptr;
+  sa.Bseq = p.B;
+  sa.Hkv = p.Hkv;
+  sa.Sk = p.Sk;
+  sa.D = 128;
+  sa.nchunks = static_cast<int>(ceil_div64(p.Sk, kSmoothChunk));
+  sa.layout = 0;
+  {
+    dim3 grid(sa.nchunks, p.B, p.Hkv);
+    if (p.dt == SKV_BF16) kmean_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(sa);
+    else kmean_partial_kernel<__half><<<grid, 256, 0, st>>>(sa);
+    kmean_finalize_kernel<<<p.B * p.Hkv, 128, 0, st>>>(sa);
+    launches += 2;
+  }
+  // codes of K - mean and of Q (+ the per-row smoothing shift)
+  QuantArgs qa;
+  qa.kmean = p.kmean;
+  qa.B = p.B;
+  qa.Hkv = p.Hkv;
+  qa.scale_log2 = p.scale * 1.4426950408889634f;
+  qa.x = p.k;
+  qa.codes = p.k8;
+  qa.scales = p.kscale;
+  qa.dq = nullptr;
+  qa.H = p.Hkv;
+  qa.S = p.Sk;
+  qa.nblk = nkb;
+  if (p.dt == SKV_BF16) quant_int8_kernel<__nv_bfloat16, false><<<dim3(nkb, p.B * p.Hkv), 256, 0, st>>>(qa);
+  else quant_int8_kernel<__half, false><<<dim3(nkb, p.B * p.Hkv), 256, 0, st>>>(qa);
+  qa.x = p.q;
+  qa.codes = p.q8;
+  qa.scales = p.qscale;
+  qa.dq = p.dq;
+  qa.H = p.Hq;
+  qa.S = p.Sq;
+  qa.nblk = nqb;
+  if (p.dt == SKV_BF16) quant_int8_kernel<__nv_bfloat16, true><<<dim3(nqb, p.B * p.Hq), 256, 0, st>>>(qa);
+  else quant_int8_kernel<__half, true><<<dim3(nqb, p.B * p.Hq), 256, 0, st>>>(qa);
+  launches += 2;
+  cudaError_t le = cudaGetLastError();
+  if (le != cudaSuccess) return le;
+  count_launches(launches);
+  // the prefill over the codes (V stays 16-bit)
+  CUtensorMap tq, tk, tv;
+  int e = make_i8_map(&tq, p.q8, p.B, p.Hq, p.Sq);
+  if (e) return e;
+  e = make_i8_map(&tk, p.k8, p.B, p.Hkv, p.Sk);
+  if (e) return e;
+  e = make_qkv_map(&tv, p.v, p.dt, SKV_HND, p.B, p.Hkv, p.Sk, 128);
+  if (e) return e;
+  PrefillArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.out = p.out;
+  a.lse = p.lse;
+  a.qscale = p.qscale;
+  a.kscale = p.kscale;
+  a.dq = p.dq;
+  a.causal = p.causal;
+  a.B = p.B;
+  a.Hq = p.Hq;
+  a.Hkv = p.Hkv;
+  a.Sq = p.Sq;
+  a.Sk = p.Sk;
+  a.layout = 0;
+  a.scale_log2 = p.scale * 1.4426950408889634f;
+  a.nqb = static_cast<int>(ceil_div64(p.Sq, kPrefillRowsPerCta));
+  const int64_t grid = static_cast<int64_t>(p.B) * p.Hq * a.nqb;
+  if (grid <= 0) return 0;
+  if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+  if (p.dt == SKV_BF16) return launch_prefill_t<128, __nv_bfloat16, true>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+  return launch_prefill_t<128, __half, true>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
 }
 
 int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int32_t* order, int32_t* offsets,

@@ -15,7 +15,8 @@
 //  * instruction descriptor (.kind::f16): D format in [4,6) (1 = f32), A format
 //    in [7,10) and B format in [10,13) (0 = f16, 1 = bf16), A / B major-ness in
 //    bits 15 / 16 (0 = K-major, 1 = MN-major), N >> 3 in [17,23), M >> 4 in
-//    [24,29).
+//    [24,29); .kind::i8 has the same fields with D format 2 = s32 and A / B
+//    format 1 = signed 8-bit.
 #pragma once
 
 #include <cstdint>
@@ -80,6 +81,25 @@ __host__ __device__ constexpr uint32_t idesc_f16(int is_bf16, int b_mn_major, in
   return (1u << 4) | (static_cast<uint32_t>(is_bf16) << 7) | (static_cast<uint32_t>(is_bf16) << 10) |
          (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor of .kind::i8: D format s32 (2 in [4,6)), A and B
+// signed 8-bit (1 in [7,10) and [10,13)), both K-major, N >> 3, M >> 4.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], signed 8-bit operands, s32 accumulate
+// (K = 32 per instruction).
+__device__ __forceinline__ void mma_ss_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 __device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
