@@ -275,9 +275,11 @@ def quantize_int8_blocks(x_rows, block: int = INT8_BLOCK) -> Tuple[np.ndarray, n
     LSE of the original logits restored afterwards.  The pages give no
     quantizer; the plainest reading, taken here: for the rows of one block,
     amax = max |x| over the block, scale = amax / 127 (a block of zeros gets
-    scale 1), code = round-half-to-even(x / scale) clamped to [-127, 127].
-    All of it in fp32 (the values are fp32: 16-bit inputs widened, or K - mean
-    in fp32), so that the integer codes are decided in the kernel's precision.
+    scale 1), code = round-half-to-even(x * (127 / amax)) clamped to
+    [-127, 127] -- one fp32 reciprocal per block and one fp32 product per
+    value (a block of zeros gets codes 0).  All of it in fp32 (the values are
+    fp32: 16-bit inputs widened, or K - mean in fp32), so that the integer
+    codes are decided in the kernel's precision.
     Returns (codes int8 [n, D], scales fp32 [ceil(n / block)]).
     """
     x32 = np.asarray(x_rows, dtype=np.float32)
@@ -289,7 +291,8 @@ def quantize_int8_blocks(x_rows, block: int = INT8_BLOCK) -> Tuple[np.ndarray, n
         blk = x32[b * block:(b + 1) * block]
         amax = np.float32(np.abs(blk).max()) if blk.size else np.float32(0.0)
         sc = np.float32(amax / np.float32(127.0)) if amax > 0 else np.float32(1.0)
-        c = np.rint(blk / sc)                       # fp32 quotient, ties to even
+        inv = np.float32(np.float32(127.0) / amax) if amax > 0 else np.float32(0.0)
+        c = np.rint(blk * inv)                      # fp32 product, ties to even
         codes[b * block:(b + 1) * block] = np.clip(c, -127, 127).astype(np.int8)
         scales[b] = sc
     return codes, scales

@@ -101,19 +101,15 @@ __device__ __forceinline__ void exp_pack_64(const float (&sv)[64], uint64_t sc2,
 
 // kI8: Q and K arrive as int8 codes (one 128-byte box per row at D = 128)
 // and S = Q K^T is an s32 .kind::i8 product; V stays 16-bit.
-// s32 logits read from TMEM (bit patterns in float registers) to exact fp32
-// values: |s| < 2^22 for int8 codes at D <= 128, so adding the bits of
-// 1.5 * 2^23 and subtracting it again is exact.
-__device__ __forceinline__ void s32_to_f32_64(float (&v)[64]) {
-  const uint64_t neg_magic = f2_pack(-12582912.0f, -12582912.0f);
+// s32 logits read from TMEM (bit patterns in float registers) as the floats
+// kMagic + s: |s| < 2^22 for int8 codes at D <= 128, so adding the bits of
+// kMagic = 1.5 * 2^23 to the integer gives that float exactly.  The kernel
+// keeps the offset and folds -kMagic * scale into the bias of its FMA, so a
+// logit costs one integer add more than in the 16-bit path.
+constexpr float kMagic = 12582912.0f;
+__device__ __forceinline__ void s32_to_magic_64(float (&v)[64]) {
 #pragma unroll
-  for (int c = 0; c < 64; c += 2) {
-    const float a0 = __int_as_float(__float_as_int(v[c]) + 0x4B400000);
-    const float a1 = __int_as_float(__float_as_int(v[c + 1]) + 0x4B400000);
-    const float2 r = f2_unpack(fadd2(f2_pack(a0, a1), neg_magic));
-    v[c] = r.x;
-    v[c + 1] = r.y;
-  }
+  for (int c = 0; c < 64; ++c) v[c] = __int_as_float(__float_as_int(v[c]) + 0x4B400000);
 }
 
 template <int D, bool kI8 = false>
@@ -528,7 +524,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tc5::ld32(s_addr + hf * 64, *reinterpret_cast<float(*)[32]>(&sh[0]));
           tc5::ld32(s_addr + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
           tc5::wait_ld();
-          if constexpr (kI8) s32_to_f32_64(sh);
+          if constexpr (kI8) s32_to_magic_64(sh);
           if (n_valid < kPfBN) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
@@ -540,7 +536,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], sh[c + e], sh[c + 8 + e]);
         }
         const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-        const float t_max = fmaf(mx, sl2, -bias_shift);
+        const float t_max = fmaf(mx, sl2, kI8 ? -fmaf(kMagic, sl2, bias_shift) : -bias_shift);
         const float m_new = fmaxf(m_run, t_max);
         const bool rescale = m_new > m_run + kPfRescaleThreshold;
         float alpha = 1.f;
@@ -573,7 +569,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // published on its own barrier, so PV can start on the first half
         // a row that has seen no key yet (causal rows before the first key)
         // keeps m = -inf: exponentiate its masked logits against 0 instead
-        const float neg_bias = -((m_run == -INFINITY ? 0.f : m_run) + bias_shift);
+        float neg_bias = -((m_run == -INFINITY ? 0.f : m_run) + bias_shift);
+        if constexpr (kI8) neg_bias = fmaf(-kMagic, sl2, neg_bias);  // the logits carry +kMagic
         const uint64_t sc2 = f2_pack(sl2, sl2);
         const uint64_t nb2 = f2_pack(neg_bias, neg_bias);
         uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -584,7 +581,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tc5::ld32(s_addr + hf * 64, *reinterpret_cast<float(*)[32]>(&sh[0]));
           tc5::ld32(s_addr + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
           tc5::wait_ld();
-          if constexpr (kI8) s32_to_f32_64(sh);
+          if constexpr (kI8) s32_to_magic_64(sh);
           if (!full_tile) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)

@@ -5,7 +5,7 @@ The codes themselves are compared too (read from the documented workspace
 sections): Q codes and scales must equal the oracle's bit for bit (the same
 fp32 operations on the same 16-bit inputs); K' = K - mean depends on the
 mean's fp32 summation order, so a K' code may differ by one where the
-oracle's x / scale lies within a hair of a rounding tie, and nowhere else."""
+oracle's x * 127 / amax lies within a hair of a rounding tie, and nowhere else."""
 import numpy as np
 import pytest
 import torch
@@ -102,8 +102,10 @@ def check_codes(d, codes):
             diff = codes["k8"][b, h].astype(int) - kc.astype(int)
             assert np.abs(diff).max() <= 1
             if np.any(diff):
-                # only where x / scale sits at a rounding tie within the mean's rounding
-                r = kp / np.repeat(ks, 128)[:kp.shape[0], None]
+                # only where x * 127 / amax sits at a rounding tie within the mean's rounding
+                amax = np.repeat([np.abs(kp[i:i + 128]).max() for i in range(0, kp.shape[0], 128)],
+                                 128)[:kp.shape[0], None].astype(np.float32)
+                r = kp * (np.float32(127.0) / amax)
                 near = np.abs(np.abs(r - np.floor(r)) - 0.5) < 1e-3
                 assert np.all(near[diff != 0])
 
