@@ -362,6 +362,11 @@ def run_ours(args, rank, world, dist):
     us_c = time_graph(lambda: skv.attn_fwd_lse(q5, k5[0], v5[0], scale, out=oc, lse=lc, causal=True), 20)
     detail["causal_prefill_h16_s4096"] = {"graph_us": round(us_c, 2),
                                           "tflops": round(FLOPS_CAUSAL_CHUNK / (us_c * 1e-6) / 1e12, 1)}
+    # INT8 Q K'^T with smooth_k on the same chunk (mean, codes and prefill: the whole call)
+    ws8 = torch.empty(skv.attn_fwd_lse_int8_workspace(1, 16, 16, 4096, 4096), dtype=torch.uint8, device=dev)
+    us_8 = time_graph(lambda: skv.attn_fwd_lse_int8(q5, k5[0], v5[0], scale, out=oc, lse=lc, workspace=ws8), 20)
+    detail["int8_smooth_prefill_h16_s4096"] = {"graph_us": round(us_8, 2),
+                                               "tflops": round(FLOPS_CFG5 / 4 / (us_8 * 1e-6) / 1e12, 1)}
     i4 = [n for n, *_r in DECODE_SHAPES].index("decode_d128_lq4_lkv32768")
     _, qd, kd, vd, scd = dec_in[i4]
     od, ld, wsd, spd = dec_buf[i4]
