@@ -601,11 +601,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
 
       // ---------------- epilogue: O / l and LSE for this thread's row
+      // O rows are staged in an idle K/V ring buffer (this tile's last K tile
+      // for tile 0, the last V tile for tile 1: both consumed once o_full
+      // fires) and then written with coalesced 16-byte stores, consecutive
+      // threads covering consecutive bytes of a row.  Chunk c of row r sits
+      // at chunk c ^ (r mod chunks), which keeps the shared-memory accesses of
+      // both phases free of bank conflicts.
+      constexpr int kRowBytes = D * 2;
+      constexpr int kChunks = kRowBytes / 16;
+      uint8_t* stg = ring + ((2 * nkv - 2 + t) % Cfg::kStages) * Cfg::kKVTileBytes;
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[t], 0, abort_flag, kErrPrefillWait));
       if (ok) {
         tc5::fence_after();
         const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;  // no key: O = 0, LSE = -inf
-        T* dst = row_valid ? out_row(qi) : nullptr;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
@@ -614,15 +622,30 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack2<T>(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
-          if (row_valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            d4[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
-            d4[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int ch = c * 4 + i;
+            *reinterpret_cast<uint4*>(stg + row * kRowBytes + ((ch ^ (row % kChunks)) * 16)) =
+                make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
         if (row_valid && a.lse != nullptr) a.lse[lse_idx(qi)] = m_run + __log2f(l_run) + delta;
+      }
+      // every warp of the tile arrives here (an aborted one too, so none waits
+      // forever); after an abort the copied rows are garbage and the device
+      // error word says so
+      named_barrier_sync(1 + t, kPfBM);
+      if (ok) {
+        const int row0 = qblk * 2 * kPfBM + t * kPfBM;
+#pragma unroll 4
+        for (int i = 0; i < kChunks; ++i) {
+          const int idx = i * kPfBM + row;
+          const int r = idx / kChunks, ch = idx % kChunks;
+          if (row0 + r < len_q) {
+            const uint4 val = *reinterpret_cast<const uint4*>(stg + r * kRowBytes + ((ch ^ (r % kChunks)) * 16));
+            *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out_row(row0 + r)) + ch * 16) = val;
+          }
+        }
       }
     }
   }
