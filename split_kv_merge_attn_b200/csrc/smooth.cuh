@@ -38,7 +38,8 @@ __device__ __forceinline__ int smooth_len(const SmoothArgs& a, int b) {
 }
 
 // grid (nchunks, Bseq, Hkv), 256 threads: (D/8) column vectors x (256/(D/8)) row lanes.
-// Every thread issues its row loads in batches of 8 before summing them.
+// Every thread issues its row loads in batches of 16 before summing them (all
+// of its rows of the chunk at D = 128: enough bytes in flight to stream K).
 template <typename T>
 __global__ void __launch_bounds__(256) kmean_partial_kernel(SmoothArgs a) {
   const int c = blockIdx.x, b = blockIdx.y, hkv = blockIdx.z;
@@ -49,17 +50,18 @@ __global__ void __launch_bounds__(256) kmean_partial_kernel(SmoothArgs a) {
   const int s0 = c * kSmoothChunk, s1 = min(len, s0 + kSmoothChunk);
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   const T* k = static_cast<const T*>(a.k);
-  // rows of this thread: s0 + rl + i * lanes; loads issued in batches of 8
-  for (int i0 = 0; i0 * lanes < kSmoothChunk; i0 += 8) {
-    uint4 u[8];
+  // rows of this thread: s0 + rl + i * lanes; loads issued in batches of 16
+  constexpr int kBatch = 16;
+  for (int i0 = 0; i0 * lanes < kSmoothChunk; i0 += kBatch) {
+    uint4 u[kBatch];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kBatch; ++i) {
       const int s = s0 + rl + (i0 + i) * lanes;
       u[i] = (s < s1) ? __ldg(reinterpret_cast<const uint4*>(k + smooth_row_off(a, b, hkv, s) + cv * 8))
                       : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kBatch; ++i) {
       const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
