@@ -48,6 +48,16 @@ DECODE_SHAPES = [  # (name, Hq, Hkv, D, Lq, Lkv)
 ]
 
 
+# The other decode shapes of the ExecuTorch split-K PR's A100 table (complete
+# graph-captured operator; D, Lq, Lkv and that table's microseconds, other
+# hardware, head counts not given there).  Timed here with workload 2's heads
+# (D128: Hq32/Hkv8) and workload 3's (D256: Hq16/Hkv4) as context lines.
+PAGES_A100_US = {("decode", 128, 1, 4096): 16.6, ("decode", 128, 1, 8192): 26.8, ("decode", 128, 1, 32768): 93.8,
+                 ("decode", 128, 4, 4096): 18.9, ("decode", 128, 4, 32768): 103.5,
+                 ("decode", 256, 1, 4096): 15.7, ("decode", 256, 1, 8192): 17.6, ("decode", 256, 1, 16384): 31.7,
+                 ("decode", 256, 1, 32768): 59.4, ("decode", 256, 4, 16384): 44.9, ("decode", 256, 4, 32768): 69.7}
+
+
 def attn_flops(rows_x_keys: int, D: int) -> int:
     """2*D FLOPs for q.k and 2*D for p*v per (query row, key) pair."""
     return 4 * D * rows_x_keys
@@ -342,7 +352,8 @@ def run_ours(args, rank, world, dist):
         us = time_graph(lambda i=i: call_decode(i), 50)
         gbs = decode_kv_bytes(Hkv, D, Lkv) / (us * 1e-6) / 1e9
         detail[name].update({"graph_us": round(us, 2), "kv_gbs": round(gbs, 1),
-                             "hbm_frac": round(gbs / peaks["hbm_gbs"], 3), "splits": dec_buf[i][3]})
+                             "hbm_frac": round(gbs / peaks["hbm_gbs"], 3), "splits": dec_buf[i][3],
+                             "pages_a100_us": PAGES_A100_US.get(("decode", D, Lq, Lkv))})
         # the single-launch variant (in-kernel merge by the last CTA of each group)
         _, q, k, v, sc = dec_in[i]
         o, l, ws, splits = dec_buf[i]
@@ -350,6 +361,24 @@ def run_ours(args, rank, world, dist):
         us_f = time_graph(lambda: skv.attn_splitkv_decode(q, k, v, sc, num_splits=splits, out=o, lse=l,
                                                           workspace=wsz, fused=True), 50)
         detail[name]["fused_graph_us"] = round(us_f, 2)
+    # the remaining shapes of the pages' decode table, graph-timed alone
+    timed = {(D, Lq, Lkv) for (_, _, _, D, Lq, Lkv) in DECODE_SHAPES}
+    for (_, D, Lq, Lkv), a100 in PAGES_A100_US.items():
+        if (D, Lq, Lkv) in timed:
+            continue
+        d = W.config2(Lq, Lkv, seed=rank) if D == 128 else W.config3(Lq, Lkv, seed=rank)
+        q, k, v, sc = d["q"].to(dev), d["k"].to(dev), d["v"].to(dev), d["scale"]
+        B, Hq, _, _ = q.shape
+        Hkv = k.shape[1]
+        splits, _ = skv.attn_splitkv_plan(B, Hq, Hkv, Lq, Lkv, D, sms, 0)
+        ws = torch.empty(max(skv.attn_splitkv_workspace(B, Hq, Lq, D, splits), 1), dtype=torch.uint8, device=dev)
+        o, l = torch.empty_like(q), torch.empty(B, Hq, Lq, dtype=torch.float32, device=dev)
+        us = time_graph(lambda: skv.attn_splitkv_decode(q, k, v, sc, num_splits=splits, out=o, lse=l, workspace=ws), 50)
+        gbs = decode_kv_bytes(Hkv, D, Lkv) / (us * 1e-6) / 1e9
+        detail[f"decode_d{D}_lq{Lq}_lkv{Lkv}"] = {"graph_us": round(us, 2), "kv_gbs": round(gbs, 1),
+                                                  "hbm_frac": round(gbs / peaks["hbm_gbs"], 3), "splits": splits,
+                                                  "pages_a100_us": a100}
+        del q, k, v, o, l, ws
     # merge_state of workload 5 alone (HBM bound)
     us_m = time_graph(lambda: skv.merge_state(o5p, l5p, "HND", out=out5, lse=lse5), 50)
     detail["merge_state_cfg5"] = {"graph_us": round(us_m, 2),
