@@ -131,6 +131,35 @@ def _need_cuda(*ts):
                 raise ValueError("tensors must be contiguous")
 
 
+def _expect(cond: bool, msg: str) -> None:
+    if not cond:
+        raise ValueError(msg)
+
+
+def _consistent(q, named, *, same_dtype=(), fp32=(), int32=()):
+    """Shape-independent consistency of the tensors of one call, checked before
+    anything reaches the library (which sees only q's dtype and the sizes read
+    off q and k): every tensor on q's device, the named 16-bit operands in q's
+    dtype, LSE buffers fp32, index arrays int32.  `named` maps names to
+    tensors (None entries are skipped)."""
+    torch = _torch()
+    for name, t in named.items():
+        if t is None:
+            continue
+        _expect(t.device == q.device, f"{name} is on {t.device}, q on {q.device}")
+        if name in same_dtype:
+            _expect(t.dtype == q.dtype, f"{name} has dtype {t.dtype}, q has {q.dtype}")
+        if name in fp32:
+            _expect(t.dtype == torch.float32, f"{name} must be float32, got {t.dtype}")
+        if name in int32:
+            _expect(t.dtype == torch.int32, f"{name} must be int32, got {t.dtype}")
+
+
+def _shape(t, shape, name: str) -> None:
+    if t is not None:
+        _expect(tuple(t.shape) == tuple(shape), f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
 def _workspace(nbytes: int, device, workspace):
     torch = _torch()
     if nbytes == 0:
@@ -203,29 +232,42 @@ def attn_fwd_lse(q, k, v, scale: Optional[float] = None, layout: str = "HND", cu
     causal: attn_fwd_lse_causal (query row i sees keys j <= i + len_k - len_q).
     """
     torch = _torch()
-    _need_cuda(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k)
+    _consistent(q, {"k": k, "v": v, "out": out, "lse": lse, "cu_seqlens_q": cu_seqlens_q,
+                    "cu_seqlens_k": cu_seqlens_k}, same_dtype=("k", "v", "out"), fp32=("lse",),
+                int32=("cu_seqlens_q", "cu_seqlens_k"))
     if layout == "TND":
         if cu_seqlens_q is None or cu_seqlens_k is None:
             raise ValueError("TND layout needs cu_seqlens_q and cu_seqlens_k")
+        _expect(q.dim() == 3 and k.dim() == 3, "TND tensors are [tokens, heads, D]")
         Tq, Hq, D = q.shape
         Tk, Hkv, _ = k.shape
         B = cu_seqlens_q.numel() - 1
+        _expect(cu_seqlens_k.numel() == B + 1, "cu_seqlens_q and cu_seqlens_k must have the same length")
         Sq, Sk = Tq, Tk
         if max_seqlen_q is None or max_seqlen_k is None:
             raise ValueError("TND layout needs max_seqlen_q and max_seqlen_k")
         lse_shape = (Hq, Tq)
+        k_shape = (Tk, Hkv, D)
     else:
+        _expect(q.dim() == 4 and k.dim() == 4, f"{layout} tensors are 4-D")
         if layout == "HND":
             B, Hq, Sq, D = q.shape
             _, Hkv, Sk, _ = k.shape
+            k_shape = (B, Hkv, Sk, D)
         elif layout == "NHD":
             B, Sq, Hq, D = q.shape
             _, Sk, Hkv, _ = k.shape
+            k_shape = (B, Sk, Hkv, D)
         else:
             raise ValueError(layout)
         max_seqlen_q = max_seqlen_q or 0
         max_seqlen_k = max_seqlen_k or 0
         lse_shape = (B, Hq, Sq)
+    _shape(k, k_shape, "k")
+    _shape(v, k_shape, "v")
+    _shape(out, q.shape, "out")
+    _shape(lse, lse_shape, "lse")
+    _need_cuda(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k)
     if scale is None:
         scale = D ** -0.5
     if out is None:
@@ -254,9 +296,15 @@ def attn_fwd_lse_int8(q, k, v, scale: Optional[float] = None, causal: bool = Fal
     """Attention with Q K'^T from INT8 codes of Q and of the smoothed K
     (dense HND, D = 128).  Returns (out, lse [B,Hq,Sq])."""
     torch = _torch()
-    _need_cuda(q, k, v, out, lse)
+    _consistent(q, {"k": k, "v": v, "out": out, "lse": lse}, same_dtype=("k", "v", "out"), fp32=("lse",))
+    _expect(q.dim() == 4 and k.dim() == 4, "HND tensors are 4-D")
     B, Hq, Sq, D = q.shape
     _, Hkv, Sk, _ = k.shape
+    _shape(k, (B, Hkv, Sk, D), "k")
+    _shape(v, (B, Hkv, Sk, D), "v")
+    _shape(out, q.shape, "out")
+    _shape(lse, (B, Hq, Sq), "lse")
+    _need_cuda(q, k, v, out, lse)
     if scale is None:
         scale = D ** -0.5
     if out is None:
@@ -292,10 +340,20 @@ def attn_splitkv_decode(q, k, v, scale: Optional[float] = None, kv_len=None, num
     zeroed once (attn_splitkv_workspace_init), one allocated here is zeroed.
     causal=True: attn_splitkv_decode_causal (row i of Lq sees the first
     kv_len - Lq + 1 + i keys); not combined with fused."""
+    if fused and causal:
+        raise ValueError("the single-launch decode has no causal variant")
     torch = _torch()
-    _need_cuda(q, k, v, out, lse, kv_len)
+    _consistent(q, {"k": k, "v": v, "out": out, "lse": lse, "kv_len": kv_len}, same_dtype=("k", "v", "out"),
+                fp32=("lse",), int32=("kv_len",))
+    _expect(q.dim() == 4 and k.dim() == 4, "decode tensors are [B, H, L, D]")
     B, Hq, Lq, D = q.shape
     _, Hkv, Lkv, _ = k.shape
+    _shape(k, (B, Hkv, Lkv, D), "k")
+    _shape(v, (B, Hkv, Lkv, D), "v")
+    _shape(out, q.shape, "out")
+    _shape(lse, (B, Hq, Lq), "lse")
+    _shape(kv_len, (B,), "kv_len")
+    _need_cuda(q, k, v, out, lse, kv_len)
     if scale is None:
         scale = D ** -0.5
     if out is None:
@@ -313,8 +371,6 @@ def attn_splitkv_decode(q, k, v, scale: Optional[float] = None, kv_len=None, num
     workspace, wbytes = _workspace(nbytes, q.device, workspace)
     if fused and fresh:
         attn_splitkv_workspace_init(workspace, stream)
-    if fused and causal:
-        raise ValueError("the single-launch decode has no causal variant")
     fn = lib().attn_splitkv_decode_fused if fused else (
         lib().attn_splitkv_decode_causal if causal else lib().attn_splitkv_decode)
     st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lkv, D, float(scale), _dtype_code(q),
@@ -330,9 +386,17 @@ def attn_splitkv_decode_static(q, k, v, scale: Optional[float] = None, kv_len=No
     per-split partials live in the library's fixed 8 MiB device array (no
     workspace).  This wrapper allocates out/lse only if they are not given."""
     torch = _torch()
-    _need_cuda(q, k, v, out, lse, kv_len)
+    _consistent(q, {"k": k, "v": v, "out": out, "lse": lse, "kv_len": kv_len}, same_dtype=("k", "v", "out"),
+                fp32=("lse",), int32=("kv_len",))
+    _expect(q.dim() == 4 and k.dim() == 4, "decode tensors are [B, H, L, D]")
     B, Hq, Lq, D = q.shape
     _, Hkv, Lkv, _ = k.shape
+    _shape(k, (B, Hkv, Lkv, D), "k")
+    _shape(v, (B, Hkv, Lkv, D), "v")
+    _shape(out, q.shape, "out")
+    _shape(lse, (B, Hq, Lq), "lse")
+    _shape(kv_len, (B,), "kv_len")
+    _need_cuda(q, k, v, out, lse, kv_len)
     if scale is None:
         scale = D ** -0.5
     if out is None:
@@ -353,17 +417,27 @@ def merge_state(o_parts, lse_parts, layout: str = "HND", out=None, lse=None, out
     """Merge P partial results.  o_parts [P,B,H,S,D] (HND), [P,B,S,H,D] (NHD)
     or [P,T,H,D] (TND); lse_parts [P,B,H,S] or [P,H,T] (fp32).  Returns (out, lse)."""
     torch = _torch()
-    _need_cuda(o_parts, lse_parts, out, lse)
+    _consistent(o_parts, {"lse_parts": lse_parts, "out": out, "lse": lse}, fp32=("lse_parts", "lse"))
     P = o_parts.shape[0]
     if layout == "HND":
+        _expect(o_parts.dim() == 5, "HND o_parts is [P, B, H, S, D]")
         _, B, H, S, D = o_parts.shape
+        lse_shape = (P, B, H, S)
     elif layout == "NHD":
+        _expect(o_parts.dim() == 5, "NHD o_parts is [P, B, S, H, D]")
         _, B, S, H, D = o_parts.shape
+        lse_shape = (P, B, H, S)
     elif layout == "TND":
+        _expect(o_parts.dim() == 4, "TND o_parts is [P, T, H, D]")
         _, S, H, D = o_parts.shape
         B = 1
+        lse_shape = (P, H, S)
     else:
         raise ValueError(layout)
+    _shape(lse_parts, lse_shape, "lse_parts")
+    _shape(out, o_parts.shape[1:], "out")
+    _shape(lse, lse_shape[1:], "lse")
+    _need_cuda(o_parts, lse_parts, out, lse)
     if out is None:
         out = torch.empty(o_parts.shape[1:], dtype=out_dtype or o_parts.dtype, device=o_parts.device)
     if return_lse and lse is None:
@@ -376,6 +450,7 @@ def merge_state(o_parts, lse_parts, layout: str = "HND", out=None, lse=None, out
     return out, lse
 
 
-__all__ = ["attn_fwd_lse", "attn_splitkv_decode", "attn_splitkv_decode_static", "merge_state", "attn_splitkv_plan", "attn_splitkv_workspace",
-           "attn_fwd_lse_workspace", "attn_varlen_plan", "device_error", "launch_count", "lib", "SkvError", "status_string",
-           "LIB_PATH", "SIGNATURES"]
+__all__ = ["attn_fwd_lse", "attn_fwd_lse_int8", "attn_splitkv_decode", "attn_splitkv_decode_static", "merge_state",
+           "attn_splitkv_plan", "attn_splitkv_workspace", "attn_splitkv_workspace_init", "attn_fwd_lse_workspace",
+           "attn_fwd_lse_int8_workspace", "attn_varlen_plan", "device_error", "launch_count", "lib", "SkvError",
+           "status_string", "LIB_PATH", "SIGNATURES"]

@@ -213,3 +213,67 @@ def test_fwd_workspace_sizes():
     # materialised K' adds one copy of K
     assert skv.attn_fwd_lse_workspace(1, 16, 16, 4096, 128, "bf16", "NHD", 2) == (
         a(16 * 128 * 4) + a(16 * 16 * 128 * 4) + a(4096 * 16 * 128 * 2))
+
+
+def test_binding_rejects_inconsistent_tensors():
+    """The Python binding checks the tensors of one call against each other
+    before anything reaches the library (which sees only q's dtype and the
+    sizes read off q and k): mismatched K/V shapes, a wrong-size output, LSE or
+    kv_len buffer, mixed dtypes.  CPU tensors suffice: these checks come before
+    the device check."""
+    import torch
+    bf = torch.bfloat16
+    q = torch.zeros(1, 4, 64, 128, dtype=bf)
+    k = torch.zeros(1, 2, 100, 128, dtype=bf)
+    v = k.clone()
+    with pytest.raises(ValueError, match="v has shape"):
+        skv.attn_fwd_lse(q, k, v[:, :, :99].contiguous(), 0.1)
+    with pytest.raises(ValueError, match="dtype"):
+        skv.attn_fwd_lse(q, k, v.half(), 0.1)
+    with pytest.raises(ValueError, match="out has shape"):
+        skv.attn_fwd_lse(q, k, v, 0.1, out=torch.zeros(1, 4, 63, 128, dtype=bf))
+    with pytest.raises(ValueError, match="lse must be float32"):
+        skv.attn_fwd_lse(q, k, v, 0.1, lse=torch.zeros(1, 4, 64, dtype=torch.float64))
+    with pytest.raises(ValueError, match="k has shape"):
+        skv.attn_fwd_lse(q, torch.zeros(1, 2, 100, 64, dtype=bf), v, 0.1)
+    # varlen
+    qt, kt = torch.zeros(10, 4, 128, dtype=bf), torch.zeros(12, 2, 128, dtype=bf)
+    cu = torch.tensor([0, 4, 10], dtype=torch.int32)
+    with pytest.raises(ValueError, match="cu_seqlens_q must be int32"):
+        skv.attn_fwd_lse(qt, kt, kt, 0.1, layout="TND", cu_seqlens_q=cu.long(), cu_seqlens_k=cu,
+                         max_seqlen_q=6, max_seqlen_k=8)
+    with pytest.raises(ValueError, match="same length"):
+        skv.attn_fwd_lse(qt, kt, kt, 0.1, layout="TND", cu_seqlens_q=cu, cu_seqlens_k=cu[:2],
+                         max_seqlen_q=6, max_seqlen_k=8)
+    with pytest.raises(ValueError, match="lse has shape"):
+        skv.attn_fwd_lse(qt, kt, kt, 0.1, layout="TND", cu_seqlens_q=cu, cu_seqlens_k=cu, max_seqlen_q=6,
+                         max_seqlen_k=8, lse=torch.zeros(10, 4))
+    # decode
+    qd = torch.zeros(1, 4, 1, 128, dtype=bf)
+    with pytest.raises(ValueError, match="kv_len has shape"):
+        skv.attn_splitkv_decode(qd, k, v, 0.1, kv_len=torch.zeros(2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="kv_len must be int32"):
+        skv.attn_splitkv_decode(qd, k, v, 0.1, kv_len=torch.zeros(1, dtype=torch.int64))
+    with pytest.raises(ValueError, match="k has shape"):
+        skv.attn_splitkv_decode(qd, torch.zeros(1, 2, 100, 64, dtype=bf), v, 0.1)
+    with pytest.raises(ValueError, match="no causal variant"):
+        skv.attn_splitkv_decode(qd, k, v, 0.1, fused=True, causal=True)
+    # int8 prefill
+    with pytest.raises(ValueError, match="v has shape"):
+        skv.attn_fwd_lse_int8(q, k, v[:, :1].contiguous(), 0.1)
+    # merge
+    o = torch.zeros(2, 1, 4, 64, 128, dtype=bf)
+    lp = torch.zeros(2, 1, 4, 64)
+    with pytest.raises(ValueError, match="lse_parts has shape"):
+        skv.merge_state(o, lp[:, :, :, :63].contiguous())
+    with pytest.raises(ValueError, match="lse_parts must be float32"):
+        skv.merge_state(o, lp.double())
+    with pytest.raises(ValueError, match="out has shape"):
+        skv.merge_state(o, lp, out=torch.zeros(1, 4, 64, 64, dtype=bf))
+    with pytest.raises(ValueError, match="lse_parts has shape"):
+        skv.merge_state(o[:, 0].contiguous(), lp, layout="TND")
+    # a consistent call made of CPU tensors stops at the device check
+    with pytest.raises(ValueError, match="CUDA"):
+        skv.attn_fwd_lse(q, k, v, 0.1)
+    with pytest.raises(ValueError, match="CUDA"):
+        skv.merge_state(o, lp)
