@@ -249,8 +249,9 @@ def smoothed_attention_rows(q, k, v, scale: float, k_smoothed: Optional[np.ndarr
     of the original logits (ARK issue: the smooth_k=True LSE lacks
     q . mean(k) * scale; adding it back fixes it).  ``k_smoothed`` may supply
     K' already rounded to a storage dtype (the kernel's reading); by default
-    K' is exact.  Parity unpinned for the ``k_smoothed`` path beyond the
-    softmax shift invariance checked in the tests.
+    K' is exact.  Both paths are pinned: the exact one by the smoothing
+    invariants, the stored-K' one against PyTorch's float64 attention over the
+    same keys and the LSE bound of the K' rounding.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)

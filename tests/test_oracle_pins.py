@@ -218,6 +218,34 @@ def test_smooth_k_invariance():
         np.testing.assert_allclose(s1, s0, atol=1e-10)
 
 
+def test_smoothed_rows_with_stored_k_prime_against_torch_float64():
+    """The materialised-K' reading (smooth_k mode 2 feeds the tensor cores K'
+    rounded to the input type): with K' supplied already rounded to bf16, the
+    oracle's smoothed O and uncorrected LSE are PyTorch's float64 SDPA and
+    logsumexp over exactly those keys; the corrected LSE adds the shift of the
+    exact mean, and the rounding of K' moves it off the exact LSE by no more
+    than the largest logit change, scale * sum|q| * max|bf16(K') - K'| / ln 2."""
+    import torch
+    d = W.config1("koff")
+    q, k, v = (O.to_f64(d[x])[0] for x in "qkv")
+    for h in range(4):
+        mu = O.kv_mean(k[h])
+        kp_exact = k[h] - mu[None]
+        kp = torch.from_numpy(kp_exact).to(torch.bfloat16).double()
+        o, lse_corr, lse_s = O.smoothed_attention_rows(q[h], k[h], v[h], d["scale"], k_smoothed=kp.numpy())
+        qt, vt = torch.from_numpy(q[h]), torch.from_numpy(v[h])
+        ref_o = torch.nn.functional.scaled_dot_product_attention(qt[None, None], kp[None, None], vt[None, None],
+                                                                 scale=d["scale"])[0, 0]
+        ref_l = torch.logsumexp(d["scale"] * (qt @ kp.T), dim=-1) / LN2
+        np.testing.assert_allclose(o, ref_o.numpy(), atol=1e-12)
+        np.testing.assert_allclose(lse_s, ref_l.numpy(), atol=1e-12)
+        np.testing.assert_allclose(lse_corr - lse_s, d["scale"] * (q[h] @ mu) / LN2, atol=1e-12)
+        _, lse_exact = O.attention_rows(q[h], k[h], v[h], d["scale"])
+        bound = d["scale"] * np.abs(q[h]).sum(-1) * np.abs(kp.numpy() - kp_exact).max() / LN2
+        assert np.all(np.abs(lse_corr - lse_exact) <= bound + 1e-12)
+        assert np.abs(lse_corr - lse_exact).max() > 0       # the rounding is visible, the bound is not vacuous
+
+
 def test_smooth_k_uncorrected_error_magnitude(golden_dir):
     """The issue prints an uncorrected smooth_k LSE error of 3.727 (16 equal
     rows, K + 0.5); over seeds the oracle's shift magnitude brackets it."""
