@@ -48,7 +48,7 @@ uint64_t launch_count() { return g_launches.load(std::memory_order_relaxed); }
 
 namespace {
 constexpr int kMaxDevices = 64;
-int g_sms[kMaxDevices] = {0};
+std::atomic<int> g_sms[kMaxDevices];  // SM count per device, 0 until first queried
 std::mutex g_mu;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -103,10 +103,13 @@ int sm_count() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0) return 0;
-  if (dev < kMaxDevices && g_sms[dev] > 0) return g_sms[dev];
+  if (dev < kMaxDevices) {
+    const int cached = g_sms[dev].load(std::memory_order_relaxed);
+    if (cached > 0) return cached;
+  }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev < kMaxDevices) g_sms[dev] = n;
+  if (dev < kMaxDevices) g_sms[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
