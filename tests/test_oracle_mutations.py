@@ -76,6 +76,35 @@ def _shift_wrong_sign(q_rows, mu, scale):
     return -scale * (np.asarray(q_rows) @ np.asarray(mu)) / math.log(2.0)
 
 
+_orig_bounds = O.split_bounds
+_orig_auto = O.auto_num_splits
+_orig_sched = O.varlen_schedule
+
+
+def _bounds_align_32(n, num_splits):
+    if n <= 0:
+        return _orig_bounds(n, num_splits)
+    C = -(-(-(-n // num_splits)) // 32) * 32          # chunk rounded to 32 keys instead of 64
+    return [min(s * C, n) for s in range(num_splits + 1)]
+
+
+def _auto_one_row_group(B, Hkv, Hq, Lq, n, num_sms, D=128):
+    return _orig_auto(B, Hkv, Hkv, 1, n, num_sms, D)   # G * Lq rows ignored: one row group per kv head
+
+
+def _sched_shortest_first(cu_seqlens_q, cu_seqlens_k, H, rows_per_cta=O.PREFILL_ROWS_PER_CTA):
+    order, offsets, items = _orig_sched(cu_seqlens_q, cu_seqlens_k, H, rows_per_cta)
+    return order[::-1], offsets, items                 # sequences taken shortest first
+
+
+def _hnd_ignores_layout(x, layout):
+    return x                                           # NHD read as if it were HND
+
+
+def _kv_mean_as_sum(k_rows):
+    return np.asarray(k_rows, dtype=np.float64).sum(axis=0)   # column sum, not mean
+
+
 PIN_TESTS = [
     lambda g: [P.test_brute_force_tiny(s) for s in range(6)],
     lambda g: [P.test_against_torch_float64(s) for s in range(3)],
@@ -92,6 +121,16 @@ PIN_TESTS = [
     lambda g: P.test_int8_quantizer_properties(),
     lambda g: P.test_int8_attention_is_exact_for_representable_inputs(),
     lambda g: P.test_int8_smoothing_is_what_makes_int8_keys_accurate(),
+    lambda g: P.test_nhd_matches_hnd(),
+    lambda g: P.test_gqa_head_mapping(),
+    lambda g: P.test_varlen_equals_dense_per_sequence(),
+    lambda g: P.test_lse_layout_adapters(),
+    lambda g: P.test_decode_equals_dense_and_kv_len(),
+    lambda g: P.test_split_bounds_partition(),
+    lambda g: P.test_split_plan_hand_values(),
+    lambda g: P.test_varlen_schedule_config4(),
+    lambda g: P.test_smooth_k_uncorrected_error_magnitude(g),
+    lambda g: P.test_smoothed_rows_with_stored_k_prime_against_torch_float64(),
 ]
 
 
@@ -115,6 +154,11 @@ def _some_pin_fails(golden_dir):
     ("causal mask aligned top-left", "causal_key_counts", _causal_counts_top_left),
     ("causal mask misses the diagonal", "causal_key_counts", _causal_counts_off_by_one),
     ("int8 scale amax / 128", "quantize_int8_blocks", _quant_scale_128),
+    ("split chunk aligned to 32 keys", "split_bounds", _bounds_align_32),
+    ("split plan ignores the query row groups", "auto_num_splits", _auto_one_row_group),
+    ("varlen work order shortest first", "varlen_schedule", _sched_shortest_first),
+    ("NHD read as HND", "_hnd", _hnd_ignores_layout),
+    ("smoothing mean is a sum", "kv_mean", _kv_mean_as_sum),
 ])
 def test_planted_mistake_is_caught(monkeypatch, golden_dir, name, attr, fn):
     monkeypatch.setattr(O, attr, fn)
