@@ -536,9 +536,27 @@ def oracle_sample(seconds_budget: float):
 
 
 def cpu_baseline(budget_s: float = 15.0):
+    """The oracle on the host cores: on all the BLAS threads it gets, and on
+    one core (BLAS limited to one thread, a shorter sample).  Each rate is also
+    turned into the seconds a whole varlen (workload 4) or chunked (workload 5)
+    problem would take at that rate: scaled from the sample, not measured."""
     flops, dt, desc = oracle_sample(budget_s)
-    return {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": desc}
+    rate = flops / dt
+    line = {"value": round(rate / 1e12, 5), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": desc,
+            "scaled_seconds": {"workload4_varlen": round(FLOPS_CFG4 / rate, 1),
+                               "workload5_chunked": round(FLOPS_CFG5 / rate, 1), "how": "scaled"}}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            f1, dt1, desc1 = oracle_sample(max(2.0, budget_s / 2))
+        r1 = f1 / dt1
+        line["one_core"] = {"value": round(r1 / 1e12, 6), "unit": "TFLOP/s", "cores": 1, "sample": desc1,
+                            "scaled_seconds": {"workload4_varlen": round(FLOPS_CFG4 / r1, 1),
+                                               "workload5_chunked": round(FLOPS_CFG5 / r1, 1), "how": "scaled"}}
+    except ImportError:
+        line["one_core"] = None
+    return line
 
 
 def run_reference(args, rank, world):

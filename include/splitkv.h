@@ -103,8 +103,13 @@ typedef enum { SKV_HND = 0, SKV_NHD = 1, SKV_TND = 2 } skv_layout;
  *   1: the smoothing is applied to the fp32 logits, s_ij - scale * q_i . mu,
  *      which is exactly K' = K - mu with no 16-bit rounding of K'.
  *   2: K' = K - mu is materialised in the input type in the workspace and used
- *      by the tensor cores; the rounding of K' to 16 bits perturbs the logits
- *      by about scale * |q| * 2^-9 * |K'| (the LSE is then accurate to that).
+ *      by the tensor cores.  The 16-bit rounding of K' perturbs every logit by
+ *      up to scale * sum_d |q_d| |K'_d| * 2^-9, so the LSE of this mode is NOT
+ *      held to the 1e-3 log2 accuracy of modes 0 and 1 against the exact
+ *      unsmoothed LSE: on randn-like inputs with K offset by 0.5 (the chunked
+ *      workload) its error is about 2e-3 log2, and it is accepted within 2e-2.
+ *      It equals, to 1e-3, the exact LSE of the logits of the rounded K'
+ *      (plus the correction).  Use mode 1 where the LSE accuracy matters.
  *   Both modes need workspace (see below); for varlen, max_seqlen_k must bound
  *   every key length.
  *
@@ -220,11 +225,20 @@ skv_status attn_splitkv_decode_causal(const void* q, const void* k, const void* 
 
 /* Split plan (host, pure integer).  For n keys, split s covers
  *   [s*C, min((s+1)*C, n)),  C = 64 * ceil(ceil(n / num_splits) / 64).
- * If requested_splits > 0 it is used as is (1..256); otherwise the count is
- * chosen so the decode grid fills num_splits SMs: B * Hkv * ceil(G*Lq/16) *
- * splits CTAs (G = Hq/Hkv) aiming at two CTAs per SM for D <= 128 and one for
- * D = 256 (the kernel's residency), keeping >= 128 keys per split, at most 256
- * splits, and none that the rounding of C would leave empty.
+ * If requested_splits > 0 it is used as is (1..256).  Otherwise, with
+ * G = Hq/Hkv and units = B * Hkv * ceil(G*Lq/16) (the decode CTAs of one
+ * split), the count is
+ *   S0 = max(1, ceil(T / units)),  T = ceil(num_sms * 1 / 1)  for D <= 128,
+ *                                  T = ceil(num_sms * 2 / 3)  for D = 256,
+ *   S1 = min(S0, max(1, ceil(n / 128)), 256)   (>= 128 keys per split),
+ *   num_splits = ceil(n / C(S1))  (n > 0; drops splits the rounding of C
+ *                                  would leave empty), else S1,
+ * i.e. about one decode CTA per SM for D <= 128 and two per three SMs for
+ * D = 256 (whose CTA keeps twice the bytes in flight).  The targets were
+ * chosen by measurement; the pages only ask for "splits sized to fill the
+ * SMs".  Examples with num_sms = 148: B=1, Hq=32, Hkv=8, Lq=1, D=128 gives 16
+ * splits at n = 4096 and 19 at n = 32768; B=1, Hq=16, Hkv=4, Lq=1, D=256
+ * gives 25 at n = 32768.
  * Writes *num_splits and, if bounds != NULL, bounds[0..num_splits] (host) with
  * split s = [bounds[s], bounds[s+1]). */
 skv_status attn_splitkv_plan(int B, int Hq, int Hkv, int Lq, int n, int D, int num_sms,
@@ -282,7 +296,12 @@ skv_status attn_splitkv_workspace_init(void* workspace, size_t workspace_bytes, 
  *   - Every call shares the one array and it keeps the last call's contents;
  *     nothing in it needs to start at zero (each call writes every partial
  *     slot it reads).  Calls that overlap on the GPU (other streams, other host
- *     threads) race on it and must be serialised by the caller. */
+ *     threads) race on it and must be serialised by the caller.
+ * Errors: the size, dtype, head-dimension and scale checks of
+ * attn_splitkv_decode come first and give its statuses; then the 8 MiB
+ * refusal; then attn_splitkv_decode's pointer checks.  A failing CUDA call
+ * (device query, address lookup) returns SKV_ERR_CUDA with the error kept for
+ * skv_last_cuda_error. */
 skv_status attn_splitkv_decode_static(const void* q, const void* k, const void* v, void* out,
                                       float* lse, int B, int Hq, int Hkv, int Lq, int Lkv, int D,
                                       float scale, skv_dtype dtype, const int32_t* kv_len,

@@ -384,7 +384,14 @@ def attn_splitkv_decode_static(q, k, v, scale: Optional[float] = None, kv_len=No
                                out=None, lse=None, return_lse: bool = True, stream=None):
     """attn_splitkv_decode for callers that cannot allocate device memory: the
     per-split partials live in the library's fixed 8 MiB device array (no
-    workspace).  This wrapper allocates out/lse only if they are not given."""
+    workspace).  This wrapper allocates out/lse only if they are not given.
+
+    The array is looked up on the device of q (made current for the call) the
+    first time a device is used: make that first call before any stream
+    capture.  Every call on a device shares the one array, so calls that
+    overlap on the GPU (several streams or host threads) race on it and must
+    be serialised by the caller.  Problems whose partials need more than
+    8 MiB raise with SKV_ERR_WORKSPACE_TOO_SMALL."""
     torch = _torch()
     _consistent(q, {"k": k, "v": v, "out": out, "lse": lse, "kv_len": kv_len}, same_dtype=("k", "v", "out"),
                 fp32=("lse",), int32=("kv_len",))
@@ -405,9 +412,10 @@ def attn_splitkv_decode_static(q, k, v, scale: Optional[float] = None, kv_len=No
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
     if not return_lse:
         lse = None
-    st = lib().attn_splitkv_decode_static(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lkv, D,
-                                          float(scale), _dtype_code(q), _ptr(kv_len), int(num_splits),
-                                          _stream(stream, q.device))
+    with torch.cuda.device(q.device):  # the scratch array is looked up on the current device
+        st = lib().attn_splitkv_decode_static(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lkv,
+                                              D, float(scale), _dtype_code(q), _ptr(kv_len), int(num_splits),
+                                              _stream(stream, q.device))
     _check(st, "attn_splitkv_decode_static")
     return out, lse
 

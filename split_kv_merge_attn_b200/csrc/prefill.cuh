@@ -41,59 +41,15 @@ constexpr int kPfBN = 128;          // keys per KV tile
 constexpr int kPfThreads = 320;
 constexpr float kPfRescaleThreshold = 8.0f;
 
-// Tuning switch (compile time).  SKV_PF_POLY_PAIRS: of every 16 pairs of
-// probabilities, this many are computed with the FMA-pipe polynomial below
-// instead of the MUFU ex2 (0 by default: measured slower on B200, where the
-// softmax is latency- rather than MUFU-bound).
-#ifndef SKV_PF_POLY_PAIRS
-#define SKV_PF_POLY_PAIRS 0
-#endif
-
-// 2^x on the FMA pipe for x in [-126, 2^22): Cody-Waite style split
-// x = n + r with n = round(x) (the 1.5 * 2^23 addition trick) and r in
-// [-1/2, 1/2], 2^r from a degree-3 polynomial fitted to minimise the maximum
-// relative error on [-1/2, 1/2] (7.5e-5; coefficients from exp2_poly_fit.py
-// beside this file), and 2^n applied by adding n to the exponent field.
-// Arguments below -126 are clamped there (result < 2^-125, i.e. 0 for every
-// sum it enters).  Used for a fraction of the softmax probabilities so the
-// MUFU exp unit is not the only one working.
-constexpr float kExp2C0 = 0.9999280729428965f;
-constexpr float kExp2C1 = 0.6932609762204822f;
-constexpr float kExp2C2 = 0.2426111270828907f;
-constexpr float kExp2C3 = 0.05517171959872975f;
-
-__device__ __forceinline__ void poly_exp2_pair(uint64_t x2, float& p0, float& p1) {
-  float2 x = f2_unpack(x2);
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const uint64_t xc = f2_pack(x.x, x.y);
-  const uint64_t y = fadd2(xc, f2_pack(12582912.f, 12582912.f));    // round(x) in the low mantissa bits
-  const uint64_t n = fadd2(y, f2_pack(-12582912.f, -12582912.f));   // round(x) as a float
-  const uint64_t r = ffma2(n, f2_pack(-1.f, -1.f), xc);              // x - round(x), exact
-  uint64_t q = ffma2(f2_pack(kExp2C3, kExp2C3), r, f2_pack(kExp2C2, kExp2C2));
-  q = ffma2(q, r, f2_pack(kExp2C1, kExp2C1));
-  q = ffma2(q, r, f2_pack(kExp2C0, kExp2C0));
-  const float2 qf = f2_unpack(q), yf = f2_unpack(y);
-  p0 = __uint_as_float(__float_as_uint(qf.x) + (__float_as_uint(yf.x) << 23));
-  p1 = __uint_as_float(__float_as_uint(qf.y) + (__float_as_uint(yf.y) << 23));
-}
-
 // Exponentiates 64 logits (32 pairs) of one row: p = 2^(s * scale_log2 + nb),
 // packs them as 16-bit pairs and accumulates the row sum in packed fp32 pairs.
-template <bool kPoly, typename T>
+template <typename T>
 __device__ __forceinline__ void exp_pack_64(const float (&sv)[64], uint64_t sc2, uint64_t nb2, uint32_t (&pk)[32],
                                             uint64_t (&ps2)[2]) {
 #pragma unroll
   for (int e = 0; e < 32; ++e) {
-    const uint64_t x2 = ffma2(f2_pack(sv[2 * e], sv[2 * e + 1]), sc2, nb2);
-    float p0, p1;
-    if (kPoly && ((e % 16) * SKV_PF_POLY_PAIRS) % 16 < SKV_PF_POLY_PAIRS) {
-      poly_exp2_pair(x2, p0, p1);
-    } else {
-      const float2 x = f2_unpack(x2);
-      p0 = ex2_approx(x.x);
-      p1 = ex2_approx(x.y);
-    }
+    const float2 x = f2_unpack(ffma2(f2_pack(sv[2 * e], sv[2 * e + 1]), sc2, nb2));
+    const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
     ps2[e & 1] = fadd2(ps2[e & 1], f2_pack(p0, p1));
     pk[e] = pack2<T>(p0, p1);
   }
@@ -574,7 +530,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint64_t sc2 = f2_pack(sl2, sl2);
         const uint64_t nb2 = f2_pack(neg_bias, neg_bias);
         uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-        const bool full_tile = n_valid >= kPfBN;  // masked tails stay on the MUFU (exact zeros)
+        const bool full_tile = n_valid >= kPfBN;
 #pragma unroll 1
         for (int hf = 0; hf < 2; ++hf) {
           float sh[64];
@@ -588,8 +544,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (hf * 64 + c >= n_valid) sh[c] = -INFINITY;
           }
           uint32_t pk[32];
-          if (full_tile) exp_pack_64<true, T>(sh, sc2, nb2, pk, ps2);
-          else exp_pack_64<false, T>(sh, sc2, nb2, pk, ps2);
+          exp_pack_64<T>(sh, sc2, nb2, pk, ps2);
           tc5::st16(s_addr + hf * 32, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
           tc5::st16(s_addr + hf * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
           tc5::wait_st();

@@ -11,14 +11,17 @@
 #include "skv_internal.h"
 
 namespace {
-
 thread_local int g_last_cuda_error = 0;
+}  // namespace
 
-skv_status cuda_status(int e) {
+skv_status skv::cuda_status(int e) {
   if (e == 0) return SKV_OK;
   g_last_cuda_error = e;
   return SKV_ERR_CUDA;
 }
+
+namespace {
+using skv::cuda_status;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 

@@ -105,6 +105,10 @@ int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partia
 
 int read_and_clear_device_error(int* code);
 
+// Maps a cudaError_t value to a status: SKV_OK for 0, else SKV_ERR_CUDA with
+// the error recorded for skv_last_cuda_error on the calling thread.
+skv_status cuda_status(int e);
+
 // Launch accounting (incremented by every successful kernel launch).
 void count_launches(int n);
 uint64_t launch_count();

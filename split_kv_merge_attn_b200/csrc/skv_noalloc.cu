@@ -15,6 +15,7 @@
 // device, with that device current, on the first call made on the device.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "skv_internal.h"
@@ -54,23 +55,29 @@ extern "C" skv_status attn_splitkv_decode_static(const void* q, const void* k, c
                                                  int B, int Hq, int Hkv, int Lq, int Lkv, int D, float scale,
                                                  skv_dtype dtype, const int32_t* kv_len, int num_splits,
                                                  skv_stream_t stream) {
-  // Size check first, so a problem that cannot fit is refused with a clear
-  // status before anything else happens.
+  // The checks that decide the split count come first (sizes, dtype, head
+  // dimension, scale), then the size refusal, so an unsupported or invalid
+  // problem gets the same status as from attn_splitkv_decode and an oversized
+  // one is refused before the scratch array is touched.  Pointer checks and
+  // the launches are those of attn_splitkv_decode, called at the end.
   if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lkv < 0 || D < 1 || Hq % Hkv != 0) return SKV_ERR_INVALID_ARG;
   if (num_splits < 0 || num_splits > skv::kSplitMax) return SKV_ERR_INVALID_ARG;
+  if (dtype != SKV_BF16 && dtype != SKV_FP16 && dtype != SKV_FP32) return SKV_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SKV_ERR_INVALID_ARG;
+  if (dtype == SKV_FP32 || (D != 64 && D != 128 && D != 256)) return SKV_ERR_UNSUPPORTED;
   int splits = num_splits;
   if (splits == 0) {
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return SKV_ERR_CUDA;
+    if (e != cudaSuccess) return skv::cuda_status(e);
     const skv_status s = attn_splitkv_plan(B, Hq, Hkv, Lq, Lkv, D, sms, 0, &splits, nullptr);
     if (s != SKV_OK) return s;
   }
   if (attn_splitkv_workspace(B, Hq, Lq, D, splits) > kStaticScratchBytes) return SKV_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
   const int e = static_scratch(&scratch);
-  if (e != 0) return SKV_ERR_CUDA;
+  if (e != 0) return skv::cuda_status(e);
   // The regular entry point does the rest (validation, launches) with the
   // static array as its workspace; it allocates nothing either.
   return attn_splitkv_decode(q, k, v, out, lse, B, Hq, Hkv, Lq, Lkv, D, scale, dtype, kv_len, splits, scratch,

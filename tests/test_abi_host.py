@@ -188,6 +188,14 @@ def test_split_plan_matches_oracle_bit_exact():
             assert s2 == req and b2 == O.split_bounds(n, req)
 
 
+def test_split_plan_examples_quoted_in_the_header():
+    """include/splitkv.h quotes the automatic plan on the decode workloads'
+    shapes with 148 SMs; the library must give exactly those counts."""
+    assert skv.attn_splitkv_plan(1, 32, 8, 1, 4096, 128, 148, 0)[0] == 16
+    assert skv.attn_splitkv_plan(1, 32, 8, 1, 32768, 128, 148, 0)[0] == 19
+    assert skv.attn_splitkv_plan(1, 16, 4, 1, 32768, 256, 148, 0)[0] == 25
+
+
 def test_varlen_plan_matches_oracle_bit_exact():
     rng = np.random.default_rng(1)
     cu = [0, 512, 1536, 3584, 7680]
