@@ -36,11 +36,20 @@ constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
 constexpr int kSplitMaxDevice = 256;   // largest num_splits (the host planner's cap)
 constexpr int kMergeStageOffset = kSplitMaxDevice * kDecodeRows * 4 + 128;  // after weights + 1/sum
 
+// Tuning switches (compile time): K/V ring depth of the decode for D = 128 and
+// D = 256 (one stage holds the K and V tiles of 64 keys).
+#ifndef SKV_DECODE_STAGES_D128
+#define SKV_DECODE_STAGES_D128 3
+#endif
+#ifndef SKV_DECODE_STAGES_D256
+#define SKV_DECODE_STAGES_D256 3
+#endif
+
 template <int D>
 struct DecodeCfg {
   static constexpr int kBoxes = D / 64;                       // 64-element column boxes per row
   static constexpr int kTileBytes = kBoxes * kDecodeKeysPerTile * 128;  // one K or V tile
-  static constexpr int kStages = (D == 64) ? 6 : 3;
+  static constexpr int kStages = (D == 64) ? 6 : (D == 128 ? SKV_DECODE_STAGES_D128 : SKV_DECODE_STAGES_D256);
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kQStride = D + 8;                      // elements; 16-byte pad per row
   static constexpr int kRingBytes = kStages * kStageBytes;

@@ -99,11 +99,93 @@ struct MergeArgs {
   int64_t n_vec;           // rows * D / 8
 };
 
+// Row-cooperative merge for many rows (the ring / chunk merge): the D/8
+// slices of one row are VPR consecutive lanes of a warp (32 / VPR rows per
+// warp), so each row's weights are computed once, not once per slice:
+//   pass 1: lane c reads the LSEs of parts c, c + VPR, ...; a shuffle max over
+//           the row's lanes gives M;
+//   pass 2: per batch of VPR parts, lane c holds w = 2^(L_{pb+c} - M) (0 for an
+//           empty part) and every lane of the row fetches the weight of the
+//           part it is about to add with a shuffle; the 16-byte O slices of up
+//           to four parts are requested together before any is used.
+// Parts of weight 0 are neither loaded nor used (their O slots may hold
+// anything).  Grid-stride over slices, so the grid can be sized to the
+// resident capacity of the GPU.
+template <typename TI, typename TO, int VPR>
+__global__ void __launch_bounds__(256) merge_rows_kernel(MergeArgs a) {
+  static_assert(32 % VPR == 0, "a row's slices stay inside one warp");
+  constexpr int kBatch = 4;
+  const TI* __restrict__ op = static_cast<const TI*>(a.o_parts);
+  const float* __restrict__ lp = a.lse_parts;
+  TO* __restrict__ out = static_cast<TO*>(a.out);
+  const int c = threadIdx.x % VPR;  // slice of the row (blockDim is a multiple of 32)
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  // the loop condition is warp-uniform (the warp's first slice), so every lane
+  // of a warp takes part in every shuffle; lanes of a row past the end only
+  // compute on empty data and store nothing
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g - lane < a.n_vec; g += stride) {
+    const bool valid = g - c < a.n_vec;  // the whole row exists
+    const int64_t row = valid ? g / VPR : 0;
+    int64_t lrow = row;
+    if (a.layout_bsh) {
+      const int h = static_cast<int>(row % a.H);
+      const int64_t bs = row / a.H;
+      const int s = static_cast<int>(bs % a.S);
+      lrow = (bs / a.S * a.H + h) * a.S + s;
+    }
+    const float* lrow_p = lp + lrow;
+    const int P = valid ? a.P : 0;
+    float m = -INFINITY;
+    for (int p = c; p < P; p += VPR) m = fmaxf(m, __ldg(lrow_p + p * a.part_stride_lse));
+#pragma unroll
+    for (int o = VPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o, VPR));
+    // if m is -inf every part of the row is empty: every weight is 0 below
+    const TI* base = op + row * a.D + c * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float wsum = 0.f;
+    for (int pb = 0; pb < a.P; pb += VPR) {
+      const int pm = pb + c;
+      const float L = pm < P ? __ldg(lrow_p + pm * a.part_stride_lse) : -INFINITY;
+      const float wl = (L == -INFINITY) ? 0.f : ex2_approx(L - m);
+      wsum += wl;
+      const int nb = min(VPR, a.P - pb);
+      for (int p0 = 0; p0 < nb; p0 += kBatch) {
+        float w[kBatch];
+        Raw8<TI> x[kBatch];
+#pragma unroll
+        for (int r = 0; r < kBatch; ++r) {  // every load of the batch is issued before any use
+          w[r] = __shfl_sync(0xffffffffu, wl, (p0 + r) % VPR, VPR);
+          if (p0 + r < nb && w[r] != 0.f) x[r].load(base + (pb + p0 + r) * a.part_stride_o);
+        }
+#pragma unroll
+        for (int r = 0; r < kBatch; ++r) {
+          if (p0 + r < nb && w[r] != 0.f) {
+            float xf[8];
+            x[r].unpack(xf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(w[r], xf[e], acc[e]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = VPR / 2; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o, VPR);
+    if (!valid) continue;
+    const float inv = (m != -INFINITY && wsum > 0.f) ? 1.0f / wsum : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] *= inv;
+    Vec8<TO>::store(out + row * a.D + c * 8, acc);
+    if (c == 0 && a.lse != nullptr) a.lse[lrow] = (m == -INFINITY) ? -INFINITY : m + __log2f(wsum);
+  }
+}
+
+// Generic many-row merge (any D that is a multiple of 8): one thread per
+// 8-element slice of one row; the loads of up to kBatch parts (LSE and O
+// slice) are issued together and merged with a running max, so a thread waits
+// for memory once per kBatch parts, not once per part.
 template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) merge_state_kernel(MergeArgs a) {
-  // one thread per 8-element slice of one row; the loads of up to kBatch parts
-  // (LSE and O slice) are issued together and merged with a running max, so a
-  // thread waits for memory once per kBatch parts, not once per part
   constexpr int kBatch = 4;
   const TI* __restrict__ op = static_cast<const TI*>(a.o_parts);
   const float* __restrict__ lp = a.lse_parts;

@@ -11,6 +11,12 @@
 
 #include "skv_internal.h"
 #include "skv_device.cuh"
+
+// Tuning switch: 1 = the row merge runs on at most the blocks the GPU holds at
+// once and strides over the rest; 0 = one block per 256 slices.
+#ifndef SKV_MERGE_RESIDENT_GRID
+#define SKV_MERGE_RESIDENT_GRID 1
+#endif
 #include "merge_state.cuh"
 #include "decode.cuh"
 #include "quant.cuh"
@@ -135,6 +141,38 @@ cudaError_t launch_parts(const MergeArgs& a, unsigned rows, cudaStream_t st, boo
 }
 }  // namespace
 
+namespace {
+// Resident 256-thread blocks of `kern` per SM (queried once per kernel).
+template <typename K>
+int resident_blocks(K kern, std::atomic<int>& cache) {
+  int v = cache.load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 256, 0) != cudaSuccess || n < 1) n = 1;
+  cache.store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Row-cooperative merge (D / 8 in {8, 16, 32}): grid = the slices' blocks, at
+// most the blocks the GPU holds at once (the kernel strides over the rest).
+template <typename TI, typename TO, int VPR>
+cudaError_t launch_rows(const MergeArgs& a, int sms, cudaStream_t st) {
+  static std::atomic<int> occ{0};
+  auto kern = merge_rows_kernel<TI, TO, VPR>;
+  const int64_t need = (a.n_vec + 255) / 256;
+  int64_t cap = need;
+#if SKV_MERGE_RESIDENT_GRID
+  cap = static_cast<int64_t>(sms) * resident_blocks(kern, occ);
+#else
+  (void)sms;
+  (void)occ;
+#endif
+  const int64_t blocks = need < cap ? need : cap;
+  kern<<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
+  return cudaSuccess;
+}
+}  // namespace
+
 int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, float* lse, int P, int B, int H,
                        int S, int D, int layout_bsh, skv_dtype parts_dt, skv_dtype out_dt,
                        int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream, bool dependent) {
@@ -161,10 +199,16 @@ int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, f
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // few rows and many parts: one CTA per row, parallel over the parts
   const bool per_row = P >= 8 && rows <= 4096 && D <= 2048 && sms > 0;
+  // many rows: the row-cooperative kernel where a row's slices fit in a warp
+  const int vpr = D / 8;
+  const bool coop = !per_row && sms > 0 && (vpr == 8 || vpr == 16 || vpr == 32);
   cudaError_t le = cudaSuccess;
 #define SKV_MERGE(TI, TO)                                                                   \
   do {                                                                                      \
     if (per_row) le = launch_parts<TI, TO>(a, static_cast<unsigned>(rows), st, dependent); \
+    else if (coop && vpr == 8) le = launch_rows<TI, TO, 8>(a, sms, st);                     \
+    else if (coop && vpr == 16) le = launch_rows<TI, TO, 16>(a, sms, st);                   \
+    else if (coop) le = launch_rows<TI, TO, 32>(a, sms, st);                                \
     else merge_state_kernel<TI, TO><<<static_cast<unsigned>(blocks), threads, 0, st>>>(a); \
   } while (0)
   if (parts_dt == SKV_FP32 && out_dt == SKV_BF16) SKV_MERGE(float, __nv_bfloat16);
