@@ -149,6 +149,37 @@ skv_status attn_fwd_lse_causal(const void* q, const void* k, const void* v, void
                                int smooth_k, void* workspace, size_t workspace_bytes,
                                skv_stream_t stream);
 
+/* attn_fwd_lse_chunks: the partial results of one query block over several
+ * KV chunks, in one launch.
+ *
+ * Chunk c is keys [chunk_bounds[c], chunk_bounds[c+1]) of every batch entry
+ * and kv head.  Its partial (O_c, LSE_c) is exactly what attn_fwd_lse gives
+ * for q against k[..., chunk c, ...], v[..., chunk c, ...] (with smooth_k,
+ * the mean is chunk c's own and LSE_c is still that of the original logits,
+ * so the partials lie on one scale).  These are the per-chunk partials that
+ * ring / chunked attention merges (ARK issue, Problem Description: chunks
+ * smoothed by their own means whose LSEs are merged; SGLang PR review thread:
+ * the per-hop merge of ring attention); merge_state of the num_chunks parts gives
+ * the attention over all Sk keys.  All chunks run in one grid, so the work of
+ * the chunks fills the GPU together instead of each leaving a partial wave.
+ *
+ * Dense layouts only (HND or NHD), non-causal.  q, k, v as attn_fwd_lse;
+ * out_parts [num_chunks, <q's shape>] in q's layout and type (part c starts
+ * c * B*Hq*Sq*D elements in); lse_parts [num_chunks, B, Hq, Sq] fp32
+ * (nullable).  chunk_bounds: HOST int32 [num_chunks + 1], chunk_bounds[0] = 0,
+ * non-decreasing, chunk_bounds[num_chunks] = Sk (empty chunks are allowed:
+ * O_c = 0, LSE_c = -inf).  1 <= num_chunks <= 64.  workspace: device,
+ * 256-byte aligned, >= attn_fwd_lse_chunks_workspace(...) bytes (0 without
+ * smooth_k).  Errors as attn_fwd_lse, and SKV_ERR_INVALID_ARG for a TND
+ * layout or invalid chunk bounds. */
+skv_status attn_fwd_lse_chunks(const void* q, const void* k, const void* v, void* out_parts,
+                               float* lse_parts, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                               float scale, skv_dtype dtype, skv_layout layout, int num_chunks,
+                               const int32_t* chunk_bounds, int smooth_k, void* workspace,
+                               size_t workspace_bytes, skv_stream_t stream);
+size_t attn_fwd_lse_chunks_workspace(int B, int Hq, int Hkv, int Sk, int D, skv_dtype dtype,
+                                     skv_layout layout, int num_chunks, int smooth_k);
+
 /* attn_fwd_lse_int8: attention with Q K'^T computed from INT8 codes.
  *
  * ARK issue, Problem Description: K is smoothed (its mean over the call's keys

@@ -10,6 +10,7 @@ library is missing or a call fails, an exception is raised.
 Entry points (same names as the C ABI):
 
 * ``attn_fwd_lse``        prefill / varlen attention, O and per-row log2 LSE
+* ``attn_fwd_lse_chunks`` the partials of several KV chunks in one launch (for merge_state)
 * ``attn_splitkv_decode`` split-KV decode (stable per-split online softmax)
 * ``merge_state``         merge partial (O, LSE) pairs of disjoint KV ranges
 * ``attn_splitkv_plan``, ``attn_splitkv_workspace``, ``attn_splitkv_workspace_init``, ``attn_fwd_lse_workspace``,
@@ -35,6 +36,10 @@ SIGNATURES = {
                               _c_int, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
     "attn_fwd_lse_causal": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_float, _c_int, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
+    "attn_fwd_lse_chunks": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                     _c_float, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _c_size, _vp]),
+    "attn_fwd_lse_chunks_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                                _c_int]),
     "attn_fwd_lse_int8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                                    _c_int, _c_int, _vp, _c_size, _vp]),
     "attn_fwd_lse_int8_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
@@ -287,6 +292,57 @@ def attn_fwd_lse(q, k, v, scale: Optional[float] = None, layout: str = "HND", cu
     return out, lse
 
 
+def attn_fwd_lse_chunks_workspace(B: int, Hq: int, Hkv: int, Sk: int, D: int, num_chunks: int, dtype: str = "bf16",
+                                  layout: str = "HND", smooth_k: int = 0) -> int:
+    return int(lib().attn_fwd_lse_chunks_workspace(B, Hq, Hkv, Sk, D, DTYPES[dtype], LAYOUTS[layout], num_chunks,
+                                                   int(smooth_k)))
+
+
+def attn_fwd_lse_chunks(q, k, v, chunk_bounds: Sequence[int], scale: Optional[float] = None, layout: str = "HND",
+                        smooth_k: int = 0, out=None, lse=None, return_lse: bool = True, workspace=None, stream=None):
+    """Partial (O, LSE) of q over each KV chunk [chunk_bounds[c], chunk_bounds[c+1])
+    in one launch (dense HND / NHD, non-causal).  Returns (out [C, *q.shape],
+    lse [C, B, Hq, Sq]); merge_state of the C parts gives attention over all keys.
+    With smooth_k each chunk is smoothed by its own mean (LSE of the original logits)."""
+    torch = _torch()
+    _consistent(q, {"k": k, "v": v, "out": out, "lse": lse}, same_dtype=("k", "v", "out"), fp32=("lse",))
+    _expect(q.dim() == 4 and k.dim() == 4, f"{layout} tensors are 4-D")
+    if layout == "HND":
+        B, Hq, Sq, D = q.shape
+        _, Hkv, Sk, _ = k.shape
+        k_shape = (B, Hkv, Sk, D)
+    elif layout == "NHD":
+        B, Sq, Hq, D = q.shape
+        _, Sk, Hkv, _ = k.shape
+        k_shape = (B, Sk, Hkv, D)
+    else:
+        raise ValueError(f"attn_fwd_lse_chunks takes HND or NHD, not {layout}")
+    C = len(chunk_bounds) - 1
+    _expect(C >= 1, "chunk_bounds needs at least two entries")
+    _shape(k, k_shape, "k")
+    _shape(v, k_shape, "v")
+    _shape(out, (C,) + tuple(q.shape), "out")
+    _shape(lse, (C, B, Hq, Sq), "lse")
+    _need_cuda(q, k, v, out, lse)
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty((C,) + tuple(q.shape), dtype=q.dtype, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((C, B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if not return_lse:
+        lse = None
+    nbytes = attn_fwd_lse_chunks_workspace(B, Hq, Hkv, Sk, D, C, {0: "bf16", 1: "fp16", 2: "fp32"}[_dtype_code(q)],
+                                           layout, smooth_k)
+    workspace, wbytes = _workspace(nbytes, q.device, workspace)
+    bounds = (ctypes.c_int32 * (C + 1))(*[int(x) for x in chunk_bounds])
+    st = lib().attn_fwd_lse_chunks(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D,
+                                   float(scale), _dtype_code(q), LAYOUTS[layout], C, bounds, int(smooth_k),
+                                   _ptr(workspace), wbytes, _stream(stream, q.device))
+    _check(st, "attn_fwd_lse_chunks")
+    return out, lse
+
+
 def attn_fwd_lse_int8_workspace(B: int, Hq: int, Hkv: int, Sq: int, Sk: int, D: int = 128) -> int:
     return int(lib().attn_fwd_lse_int8_workspace(B, Hq, Hkv, Sq, Sk, D))
 
@@ -458,7 +514,7 @@ def merge_state(o_parts, lse_parts, layout: str = "HND", out=None, lse=None, out
     return out, lse
 
 
-__all__ = ["attn_fwd_lse", "attn_fwd_lse_int8", "attn_splitkv_decode", "attn_splitkv_decode_static", "merge_state",
+__all__ = ["attn_fwd_lse", "attn_fwd_lse_chunks", "attn_fwd_lse_chunks_workspace", "attn_fwd_lse_int8", "attn_splitkv_decode", "attn_splitkv_decode_static", "merge_state",
            "attn_splitkv_plan", "attn_splitkv_workspace", "attn_splitkv_workspace_init", "attn_fwd_lse_workspace",
            "attn_fwd_lse_int8_workspace", "attn_varlen_plan", "device_error", "launch_count", "lib", "SkvError",
            "status_string", "LIB_PATH", "SIGNATURES"]

@@ -10,6 +10,8 @@
 // row (parallel over rows x D) and requests all of its parts at once.
 #pragma once
 
+#include <type_traits>
+
 #include "skv_device.cuh"
 
 namespace skv {
@@ -99,85 +101,68 @@ struct MergeArgs {
   int64_t n_vec;           // rows * D / 8
 };
 
-// Row-cooperative merge for many rows (the ring / chunk merge): the D/8
-// slices of one row are VPR consecutive lanes of a warp (32 / VPR rows per
-// warp), so each row's weights are computed once, not once per slice:
-//   pass 1: lane c reads the LSEs of parts c, c + VPR, ...; a shuffle max over
-//           the row's lanes gives M;
-//   pass 2: per batch of VPR parts, lane c holds w = 2^(L_{pb+c} - M) (0 for an
-//           empty part) and every lane of the row fetches the weight of the
-//           part it is about to add with a shuffle; the 16-byte O slices of up
-//           to four parts are requested together before any is used.
-// Parts of weight 0 are neither loaded nor used (their O slots may hold
-// anything).  Grid-stride over slices, so the grid can be sized to the
-// resident capacity of the GPU.
-template <typename TI, typename TO, int VPR>
+// Many-row merge (the ring / chunk merge) for D / 8 = VPR slices per row: one
+// thread per 8-element slice; the LSEs and O slices of up to kBatch parts are
+// all requested before any is used (one memory round trip per batch), then
+// the batch's max is taken first and each part gets one approximate exp2 (no
+// running-max chain inside a batch).  Row arithmetic is 32-bit where the slice
+// count allows it.  A part whose LSE is -inf carries no weight and its O slot
+// (which may hold anything) is not used.
+template <typename TI, typename TO, int VPR, bool kWide>
 __global__ void __launch_bounds__(256) merge_rows_kernel(MergeArgs a) {
-  static_assert(32 % VPR == 0, "a row's slices stay inside one warp");
   constexpr int kBatch = 4;
   const TI* __restrict__ op = static_cast<const TI*>(a.o_parts);
   const float* __restrict__ lp = a.lse_parts;
   TO* __restrict__ out = static_cast<TO*>(a.out);
-  const int c = threadIdx.x % VPR;  // slice of the row (blockDim is a multiple of 32)
-  const int lane = threadIdx.x & 31;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  // the loop condition is warp-uniform (the warp's first slice), so every lane
-  // of a warp takes part in every shuffle; lanes of a row past the end only
-  // compute on empty data and store nothing
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g - lane < a.n_vec; g += stride) {
-    const bool valid = g - c < a.n_vec;  // the whole row exists
-    const int64_t row = valid ? g / VPR : 0;
-    int64_t lrow = row;
-    if (a.layout_bsh) {
-      const int h = static_cast<int>(row % a.H);
-      const int64_t bs = row / a.H;
-      const int s = static_cast<int>(bs % a.S);
-      lrow = (bs / a.S * a.H + h) * a.S + s;
-    }
-    const float* lrow_p = lp + lrow;
-    const int P = valid ? a.P : 0;
-    float m = -INFINITY;
-    for (int p = c; p < P; p += VPR) m = fmaxf(m, __ldg(lrow_p + p * a.part_stride_lse));
-#pragma unroll
-    for (int o = VPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o, VPR));
-    // if m is -inf every part of the row is empty: every weight is 0 below
-    const TI* base = op + row * a.D + c * 8;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    float wsum = 0.f;
-    for (int pb = 0; pb < a.P; pb += VPR) {
-      const int pm = pb + c;
-      const float L = pm < P ? __ldg(lrow_p + pm * a.part_stride_lse) : -INFINITY;
-      const float wl = (L == -INFINITY) ? 0.f : ex2_approx(L - m);
-      wsum += wl;
-      const int nb = min(VPR, a.P - pb);
-      for (int p0 = 0; p0 < nb; p0 += kBatch) {
-        float w[kBatch];
-        Raw8<TI> x[kBatch];
-#pragma unroll
-        for (int r = 0; r < kBatch; ++r) {  // every load of the batch is issued before any use
-          w[r] = __shfl_sync(0xffffffffu, wl, (p0 + r) % VPR, VPR);
-          if (p0 + r < nb && w[r] != 0.f) x[r].load(base + (pb + p0 + r) * a.part_stride_o);
-        }
-#pragma unroll
-        for (int r = 0; r < kBatch; ++r) {
-          if (p0 + r < nb && w[r] != 0.f) {
-            float xf[8];
-            x[r].unpack(xf);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(w[r], xf[e], acc[e]);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int o = VPR / 2; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o, VPR);
-    if (!valid) continue;
-    const float inv = (m != -INFINITY && wsum > 0.f) ? 1.0f / wsum : 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] *= inv;
-    Vec8<TO>::store(out + row * a.D + c * 8, acc);
-    if (c == 0 && a.lse != nullptr) a.lse[lrow] = (m == -INFINITY) ? -INFINITY : m + __log2f(wsum);
+  using Idx = typename std::conditional<kWide, int64_t, int32_t>::type;
+  const Idx g = static_cast<Idx>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (g >= a.n_vec) return;
+  const Idx row = g / VPR;
+  const int c = static_cast<int>(g % VPR);
+  Idx lrow = row;
+  if (a.layout_bsh) {
+    const Idx h = row % a.H;
+    const Idx bs = row / a.H;
+    lrow = (bs / a.S * a.H + h) * a.S + bs % a.S;
   }
+  const TI* base = op + static_cast<int64_t>(row) * a.D + c * 8;
+  const float* lbase = lp + lrow;
+  float m = -INFINITY, W = 0.f;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int p0 = 0; p0 < a.P; p0 += kBatch) {
+    float L[kBatch];
+    Raw8<TI> x[kBatch];
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      const int p = p0 + r;
+      L[r] = (p < a.P) ? __ldg(lbase + p * a.part_stride_lse) : -INFINITY;
+      if (p < a.P) x[r].load(base + p * a.part_stride_o);
+    }
+    float mb = m;
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) mb = fmaxf(mb, L[r]);
+    if (mb == -INFINITY) continue;          // every part so far is empty
+    const float sc = ex2_approx(m - mb);    // 0 while m is -inf
+    W *= sc;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] *= sc;
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      if (L[r] == -INFINITY) continue;      // an empty part: its O slot is not used
+      const float w = ex2_approx(L[r] - mb);
+      float xf[8];
+      x[r].unpack(xf);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, xf[e], acc[e]);
+      W += w;
+    }
+    m = mb;
+  }
+  const float inv = (m != -INFINITY && W > 0.f) ? 1.0f / W : 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] *= inv;
+  Vec8<TO>::store(out + static_cast<int64_t>(row) * a.D + c * 8, acc);
+  if (c == 0 && a.lse != nullptr) a.lse[lrow] = (m == -INFINITY) ? -INFINITY : m + __log2f(W);
 }
 
 // Generic many-row merge (any D that is a multiple of 8): one thread per

@@ -110,6 +110,11 @@ struct PrefillArgs {
   int layout;           // 0 HND, 1 NHD, 2 TND
   int causal;           // 1: row i of a sequence sees keys j <= i + len_k - len_q
   float scale_log2;
+  // Multi-chunk dense call: KV chunk c is keys [kvb[c], kvb[c+1]) of every
+  // batch entry; its partial O and LSE go to out / lse + c * the size of one
+  // output (nchunks = 1: the whole key range, one output).
+  int nchunks;
+  int kvb[kMaxKvChunks + 1];
 };
 
 template <int D, typename T, bool kI8 = false>
@@ -142,6 +147,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   // ---------------- work item
   int b, h, qblk, len_q, len_k, q_row0, k_row0, bcoord;
+  int chunk = 0;  // KV chunk of a multi-chunk call
   if (a.layout == 2) {
     const int item = blockIdx.x;
     if (item >= a.offsets[a.B]) return;
@@ -168,7 +174,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     k_row0 = a.cu_k[b];
     bcoord = 0;
   } else {
-    const int item = blockIdx.x;
+    int item = blockIdx.x;
+    if (a.nchunks > 1) {  // chunk-major: the CTAs running together share one chunk's K/V
+      const int per = a.B * a.Hq * a.nqb;
+      chunk = item / per;
+      item -= chunk * per;
+    }
     if (a.causal) {
       // causal work grows with the block index: longest blocks (of every
       // batch and head) first, so the grid runs longest-processing-time first
@@ -182,11 +193,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       b = item / (a.nqb * a.Hq);
     }
     len_q = a.Sq;
-    len_k = a.Sk;
+    len_k = a.kvb[chunk + 1] - a.kvb[chunk];
     q_row0 = qblk * 2 * kPfBM;
-    k_row0 = 0;
+    k_row0 = a.kvb[chunk];
     bcoord = b;
   }
+  // smooth_k statistics are per (batch or sequence, chunk): index `seq` of
+  // nseq such ranges
+  const int seq = b * a.nchunks + chunk;
+  const int nseq = a.B * a.nchunks;
   const int hkv = h / G;
   const int rows_here = min(2 * kPfBM, len_q - qblk * 2 * kPfBM);
   const int nt = rows_here > kPfBM ? 2 : 1;
@@ -198,17 +213,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int kv_end = a.causal ? min(max(qblk * 2 * kPfBM + rows_here + causal_off, 0), len_k) : len_k;
   const int nkv = (kv_end + kPfBN - 1) / kPfBN;
 
-  // output addressing for query row qi (index inside the sequence)
+  // output addressing for query row qi (index inside the sequence); the rows
+  // of chunk c start c outputs further
+  const int64_t chunk_rows = static_cast<int64_t>(chunk) * a.B * a.Hq * a.Sq;
   auto out_row = [&](int qi) -> T* {
     int64_t r;
     if (a.layout == 0) r = (static_cast<int64_t>(b) * a.Hq + h) * a.Sq + qi;
     else if (a.layout == 1) r = (static_cast<int64_t>(b) * a.Sq + qi) * a.Hq + h;
     else r = static_cast<int64_t>(a.cu_q[b] + qi) * a.Hq + h;
-    return static_cast<T*>(a.out) + r * D;
+    return static_cast<T*>(a.out) + (chunk_rows + r) * D;
   };
   auto lse_idx = [&](int qi) -> int64_t {
     if (a.layout == 2) return static_cast<int64_t>(h) * a.Sq + a.cu_q[b] + qi;
-    return (static_cast<int64_t>(b) * a.Hq + h) * a.Sq + qi;
+    return chunk_rows + (static_cast<int64_t>(b) * a.Hq + h) * a.Sq + qi;
   };
 
   if (nkv == 0) {
@@ -414,13 +431,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int nch = (len_k + 255) / 256;
             float sum = 0.f;
             for (int c = 0; c < nch; ++c)
-              sum += __ldg(a.kpartial + ((static_cast<int64_t>(c) * a.B + b) * a.Hkv + hkv) * D + row);
+              sum += __ldg(a.kpartial + ((static_cast<int64_t>(c) * nseq + seq) * a.Hkv + hkv) * D + row);
             mu_s[row] = sum / static_cast<float>(len_k);
           }
           named_barrier_sync(1 + t, kPfBM);
           mu = mu_s;
         } else {
-          mu = a.kmean + (static_cast<int64_t>(b) * a.Hkv + hkv) * D;
+          mu = a.kmean + (static_cast<int64_t>(seq) * a.Hkv + hkv) * D;
         }
         ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, kErrPrefillWait));
         if (ok) {

@@ -34,7 +34,10 @@ struct FwdWorkspace {
   size_t order = 0, offsets = 0, kmean = 0, partial = 0, kprime = 0, total = 0;
 };
 
-FwdWorkspace fwd_workspace(int B, int Hkv, int Sk, int D, skv_layout layout, int smooth_k) {
+// nranges: key ranges per batch entry with their own smoothing mean (the
+// chunks of a multi-chunk call; 1 otherwise).  The per-256-key column sums
+// are sized for ranges as long as Sk.
+FwdWorkspace fwd_workspace(int B, int Hkv, int Sk, int D, skv_layout layout, int smooth_k, int nranges = 1) {
   FwdWorkspace w;
   size_t off = 0;
   if (layout == SKV_TND) {
@@ -45,10 +48,11 @@ FwdWorkspace fwd_workspace(int B, int Hkv, int Sk, int D, skv_layout layout, int
   }
   if (smooth_k) {
     const size_t nchunks = static_cast<size_t>(skv::ceil_div64(Sk, 256));
+    const size_t ranges = static_cast<size_t>(B) * nranges;
     w.kmean = off;
-    off += skv::align256(static_cast<size_t>(B) * Hkv * D * 4);
+    off += skv::align256(ranges * Hkv * D * 4);
     w.partial = off;
-    off += skv::align256(nchunks * B * Hkv * D * 4);
+    off += skv::align256(nchunks * ranges * Hkv * D * 4);
     if (smooth_k == 2) {
       const size_t rows = layout == SKV_TND ? static_cast<size_t>(Sk) : static_cast<size_t>(B) * Sk;
       w.kprime = off;
@@ -188,7 +192,7 @@ skv_status fwd_lse_impl(const void* q, const void* k, const void* v, void* out, 
                         int Sq, int Sk, int D, float scale, skv_dtype dtype, skv_layout layout,
                         const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int max_seqlen_q,
                         int max_seqlen_k, int smooth_k, void* workspace, size_t workspace_bytes,
-                        skv_stream_t stream, int causal) {
+                        skv_stream_t stream, int causal, int nchunks = 1, const int32_t* kv_bounds = nullptr) {
   // ---- validation (no device work before it passes)
   if (q == nullptr || out == nullptr) return SKV_ERR_INVALID_ARG;
   if ((k == nullptr || v == nullptr) && Sk != 0) return SKV_ERR_INVALID_ARG;
@@ -213,7 +217,22 @@ skv_status fwd_lse_impl(const void* q, const void* k, const void* v, void* out, 
   // TMA extents and int32 coordinates
   const int64_t rows_q = varlen ? Sq : static_cast<int64_t>(Sq);
   if (rows_q > (int64_t(1) << 31) - 512 || Sk > (1 << 30)) return SKV_ERR_UNSUPPORTED;
-  const FwdWorkspace ws = fwd_workspace(B, Hkv, Sk, D, layout, smooth_k);
+  if (nchunks < 1 || nchunks > skv::kMaxKvChunks) return SKV_ERR_INVALID_ARG;
+  int max_chunk = Sk;
+  if (nchunks > 1) {
+    if (varlen || causal || kv_bounds == nullptr) return SKV_ERR_INVALID_ARG;
+    if (kv_bounds[0] != 0 || kv_bounds[nchunks] != Sk) return SKV_ERR_INVALID_ARG;
+    max_chunk = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      if (kv_bounds[c + 1] < kv_bounds[c]) return SKV_ERR_INVALID_ARG;
+      max_chunk = std::max(max_chunk, kv_bounds[c + 1] - kv_bounds[c]);
+    }
+    // every chunk's partial is one output's worth of rows further
+    if (static_cast<int64_t>(nchunks) * B * Hq * ((Sq + skv::kPrefillRowsPerCta - 1) / skv::kPrefillRowsPerCta) >
+        0x7fffffff)
+      return SKV_ERR_UNSUPPORTED;
+  }
+  const FwdWorkspace ws = fwd_workspace(B, Hkv, Sk, D, layout, smooth_k, nchunks);
   if (workspace_bytes < ws.total) return SKV_ERR_WORKSPACE_TOO_SMALL;
   if (ws.total > 0 && (workspace == nullptr || !aligned(workspace, 256))) return SKV_ERR_INVALID_ARG;
   if (Sq == 0) return SKV_OK;  // nothing to compute
@@ -237,6 +256,8 @@ skv_status fwd_lse_impl(const void* q, const void* k, const void* v, void* out, 
   p.dt = dtype;
   p.layout = layout;
   p.causal = causal ? 1 : 0;
+  p.nchunks = nchunks;
+  p.kv_bounds = nchunks > 1 ? kv_bounds : nullptr;
   if (varlen) {
     p.cu_q = cu_seqlens_q;
     p.cu_k = cu_seqlens_k;
@@ -250,9 +271,9 @@ skv_status fwd_lse_impl(const void* q, const void* k, const void* v, void* out, 
     float* kmean = reinterpret_cast<float*>(wsb + ws.kmean);
     float* partial = reinterpret_cast<float*>(wsb + ws.partial);
     void* kprime = smooth_k == 2 ? static_cast<void*>(wsb + ws.kprime) : nullptr;
-    const int max_len = varlen ? max_seqlen_k : Sk;
+    const int max_len = varlen ? max_seqlen_k : max_chunk;
     int e = skv::launch_smooth_k(k, kprime, kmean, partial, varlen ? cu_seqlens_k : nullptr, B, Hkv, Sk, max_len,
-                                 D, dtype, layout, stream);
+                                 D, dtype, layout, stream, nchunks, nchunks > 1 ? kv_bounds : nullptr);
     if (e) return cuda_status(e);
     if (smooth_k == 1) {
       p.kpartial = partial;   // the prefill kernel sums these into the mean itself
@@ -282,6 +303,29 @@ skv_status attn_fwd_lse_causal(const void* q, const void* k, const void* v, void
                                skv_stream_t stream) {
   return fwd_lse_impl(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, dtype, layout, cu_seqlens_q, cu_seqlens_k,
                       max_seqlen_q, max_seqlen_k, smooth_k, workspace, workspace_bytes, stream, 1);
+}
+
+size_t attn_fwd_lse_chunks_workspace(int B, int Hq, int Hkv, int Sk, int D, skv_dtype dtype, skv_layout layout,
+                                     int num_chunks, int smooth_k) {
+  (void)Hq;
+  (void)dtype;
+  if (B < 1 || Hkv < 1 || Sk < 0 || D < 1 || smooth_k < 0 || smooth_k > 2) return 0;
+  if (layout != SKV_HND && layout != SKV_NHD) return 0;
+  if (num_chunks < 1 || num_chunks > skv::kMaxKvChunks) return 0;
+  return fwd_workspace(B, Hkv, Sk, D, layout, smooth_k, num_chunks).total;
+}
+
+skv_status attn_fwd_lse_chunks(const void* q, const void* k, const void* v, void* out_parts, float* lse_parts, int B,
+                               int Hq, int Hkv, int Sq, int Sk, int D, float scale, skv_dtype dtype,
+                               skv_layout layout, int num_chunks, const int32_t* chunk_bounds, int smooth_k,
+                               void* workspace, size_t workspace_bytes, skv_stream_t stream) {
+  if (layout != SKV_HND && layout != SKV_NHD) return SKV_ERR_INVALID_ARG;
+  if (num_chunks < 1 || num_chunks > skv::kMaxKvChunks || chunk_bounds == nullptr) return SKV_ERR_INVALID_ARG;
+  if (chunk_bounds[0] != 0 || chunk_bounds[num_chunks] != Sk) return SKV_ERR_INVALID_ARG;
+  for (int c = 0; c < num_chunks; ++c)
+    if (chunk_bounds[c + 1] < chunk_bounds[c]) return SKV_ERR_INVALID_ARG;
+  return fwd_lse_impl(q, k, v, out_parts, lse_parts, B, Hq, Hkv, Sq, Sk, D, scale, dtype, layout, nullptr, nullptr, 0,
+                      0, smooth_k, workspace, workspace_bytes, stream, 0, num_chunks, chunk_bounds);
 }
 
 // ------------------------------------------------------------------ int8 prefill

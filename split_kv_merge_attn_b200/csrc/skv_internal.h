@@ -30,6 +30,8 @@ constexpr int kSplitMax = 256;
 constexpr int kCtasPerSmNum = 1, kCtasPerSmDen = 1;
 constexpr int kCtasPerSmD256Num = 2, kCtasPerSmD256Den = 3;
 constexpr int kDecodeRowsPerCta = 16;
+// Largest number of KV chunks of one multi-chunk prefill call.
+constexpr int kMaxKvChunks = 64;
 constexpr int kPrefillRowsPerCta = 256;
 
 inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -68,6 +70,8 @@ struct PrefillLaunch {
   float scale;
   skv_dtype dt;
   skv_layout layout;
+  int nchunks;               // dense: KV chunks (1 = the whole key range)
+  const int32_t* kv_bounds;  // host [nchunks + 1] chunk bounds, or null when nchunks == 1
 };
 int launch_prefill(const PrefillLaunch& p, skv_stream_t stream);
 
@@ -100,8 +104,11 @@ int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, 
 // smooth_k prepass: fp32 per-256-key column sums of K for each (batch or
 // sequence, kv head) into `partial`; if k_smoothed != null also the mean
 // kmean [B, Hkv, D] and K' = K - mean rounded to the input type.
+// Dense multi-chunk calls pass kv_ranges > 1 chunks per batch entry with host
+// bounds kv_bounds[kv_ranges + 1]; every mean is then per (batch, chunk).
 int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partial, const int32_t* cu_k, int B,
-                    int Hkv, int Sk, int max_len, int D, skv_dtype dt, skv_layout layout, skv_stream_t stream);
+                    int Hkv, int Sk, int max_len, int D, skv_dtype dt, skv_layout layout, skv_stream_t stream,
+                    int kv_ranges = 1, const int32_t* kv_bounds = nullptr);
 
 int read_and_clear_device_error(int* code);
 

@@ -12,11 +12,6 @@
 #include "skv_internal.h"
 #include "skv_device.cuh"
 
-// Tuning switch: 1 = the row merge runs on at most the blocks the GPU holds at
-// once and strides over the rest; 0 = one block per 256 slices.
-#ifndef SKV_MERGE_RESIDENT_GRID
-#define SKV_MERGE_RESIDENT_GRID 1
-#endif
 #include "merge_state.cuh"
 #include "decode.cuh"
 #include "quant.cuh"
@@ -142,33 +137,15 @@ cudaError_t launch_parts(const MergeArgs& a, unsigned rows, cudaStream_t st, boo
 }  // namespace
 
 namespace {
-// Resident 256-thread blocks of `kern` per SM (queried once per kernel).
-template <typename K>
-int resident_blocks(K kern, std::atomic<int>& cache) {
-  int v = cache.load(std::memory_order_relaxed);
-  if (v > 0) return v;
-  int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 256, 0) != cudaSuccess || n < 1) n = 1;
-  cache.store(n, std::memory_order_relaxed);
-  return n;
-}
-
-// Row-cooperative merge (D / 8 in {8, 16, 32}): grid = the slices' blocks, at
-// most the blocks the GPU holds at once (the kernel strides over the rest).
+// Many-row merge with D / 8 = VPR: one thread per slice, one block per 256
+// slices; 32-bit row arithmetic when the slice count fits.
 template <typename TI, typename TO, int VPR>
-cudaError_t launch_rows(const MergeArgs& a, int sms, cudaStream_t st) {
-  static std::atomic<int> occ{0};
-  auto kern = merge_rows_kernel<TI, TO, VPR>;
-  const int64_t need = (a.n_vec + 255) / 256;
-  int64_t cap = need;
-#if SKV_MERGE_RESIDENT_GRID
-  cap = static_cast<int64_t>(sms) * resident_blocks(kern, occ);
-#else
-  (void)sms;
-  (void)occ;
-#endif
-  const int64_t blocks = need < cap ? need : cap;
-  kern<<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
+cudaError_t launch_rows(const MergeArgs& a, cudaStream_t st) {
+  const int64_t blocks = (a.n_vec + 255) / 256;
+  if (a.n_vec < (int64_t(1) << 31) - 256 && static_cast<int64_t>(a.B) * a.H * a.S * a.D < (int64_t(1) << 31))
+    merge_rows_kernel<TI, TO, VPR, false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
+  else
+    merge_rows_kernel<TI, TO, VPR, true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
   return cudaSuccess;
 }
 }  // namespace
@@ -199,16 +176,16 @@ int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, f
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // few rows and many parts: one CTA per row, parallel over the parts
   const bool per_row = P >= 8 && rows <= 4096 && D <= 2048 && sms > 0;
-  // many rows: the row-cooperative kernel where a row's slices fit in a warp
+  // many rows, D in {64, 128, 256}: the kernel specialised on the slices per row
   const int vpr = D / 8;
-  const bool coop = !per_row && sms > 0 && (vpr == 8 || vpr == 16 || vpr == 32);
+  const bool coop = !per_row && (vpr == 8 || vpr == 16 || vpr == 32);
   cudaError_t le = cudaSuccess;
 #define SKV_MERGE(TI, TO)                                                                   \
   do {                                                                                      \
     if (per_row) le = launch_parts<TI, TO>(a, static_cast<unsigned>(rows), st, dependent); \
-    else if (coop && vpr == 8) le = launch_rows<TI, TO, 8>(a, sms, st);                     \
-    else if (coop && vpr == 16) le = launch_rows<TI, TO, 16>(a, sms, st);                   \
-    else if (coop) le = launch_rows<TI, TO, 32>(a, sms, st);                                \
+    else if (coop && vpr == 8) le = launch_rows<TI, TO, 8>(a, st);                          \
+    else if (coop && vpr == 16) le = launch_rows<TI, TO, 16>(a, st);                        \
+    else if (coop) le = launch_rows<TI, TO, 32>(a, st);                                     \
     else merge_state_kernel<TI, TO><<<static_cast<unsigned>(blocks), threads, 0, st>>>(a); \
   } while (0)
   if (parts_dt == SKV_FP32 && out_dt == SKV_BF16) SKV_MERGE(float, __nv_bfloat16);
@@ -366,6 +343,13 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   a.Sk = p.Sk;
   a.layout = varlen ? 2 : (p.layout == SKV_HND ? 0 : 1);
   a.scale_log2 = p.scale * 1.4426950408889634f;
+  const int nch = (varlen || p.nchunks < 1) ? 1 : p.nchunks;
+  if (nch > kMaxKvChunks || (nch > 1 && p.kv_bounds == nullptr)) return cudaErrorInvalidValue;
+  a.nchunks = nch;
+  a.kvb[0] = 0;
+  a.kvb[1] = p.Sk;
+  if (nch > 1)
+    for (int c = 0; c <= nch; ++c) a.kvb[c] = p.kv_bounds[c];
   int64_t grid;
   if (varlen) {
     // upper bound on sum_b ceil(len_q(b) / 256); surplus CTAs exit at once
@@ -373,7 +357,7 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
     grid = static_cast<int64_t>(p.Hq) * (ceil_div64(p.Sq, kPrefillRowsPerCta) + p.B);
   } else {
     a.nqb = static_cast<int>(ceil_div64(p.Sq, kPrefillRowsPerCta));
-    grid = static_cast<int64_t>(p.B) * p.Hq * a.nqb;
+    grid = static_cast<int64_t>(nch) * p.B * p.Hq * a.nqb;
   }
   if (grid <= 0) return 0;
   if (grid > 0x7fffffff) return cudaErrorInvalidValue;
@@ -406,6 +390,9 @@ int launch_prefill_int8(const Int8PrefillLaunch& p, skv_stream_t stream) {
   sa.D = 128;
   sa.nchunks = static_cast<int>(ceil_div64(p.Sk, kSmoothChunk));
   sa.layout = 0;
+  sa.kv_ranges = 1;
+  sa.kvb[0] = 0;
+  sa.kvb[1] = p.Sk;
   {
     dim3 grid(sa.nchunks, p.B, p.Hkv);
     if (p.dt == SKV_BF16) kmean_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(sa);
@@ -464,6 +451,9 @@ int launch_prefill_int8(const Int8PrefillLaunch& p, skv_stream_t stream) {
   a.Sk = p.Sk;
   a.layout = 0;
   a.scale_log2 = p.scale * 1.4426950408889634f;
+  a.nchunks = 1;
+  a.kvb[0] = 0;
+  a.kvb[1] = p.Sk;
   a.nqb = static_cast<int>(ceil_div64(p.Sq, kPrefillRowsPerCta));
   const int64_t grid = static_cast<int64_t>(p.B) * p.Hq * a.nqb;
   if (grid <= 0) return 0;
@@ -484,30 +474,37 @@ int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, 
 // ------------------------------------------------------------ smooth_k
 
 int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partial, const int32_t* cu_k, int B,
-                    int Hkv, int Sk, int max_len, int D, skv_dtype dt, skv_layout layout, skv_stream_t stream) {
+                    int Hkv, int Sk, int max_len, int D, skv_dtype dt, skv_layout layout, skv_stream_t stream,
+                    int kv_ranges, const int32_t* kv_bounds) {
   SmoothArgs a;
   a.k = k;
   a.k_out = k_smoothed;
   a.partial = partial;
   a.kmean = kmean;
   a.cu_k = cu_k;
-  a.Bseq = B;
   a.Hkv = Hkv;
   a.Sk = Sk;
   a.D = D;
-  a.nchunks = static_cast<int>(ceil_div64(max_len, kSmoothChunk));
   a.layout = layout == SKV_HND ? 0 : (layout == SKV_NHD ? 1 : 2);
+  a.kv_ranges = (layout == SKV_TND || kv_ranges < 1) ? 1 : kv_ranges;
+  if (a.kv_ranges > kMaxKvChunks || (a.kv_ranges > 1 && kv_bounds == nullptr)) return cudaErrorInvalidValue;
+  a.kvb[0] = 0;
+  a.kvb[1] = Sk;
+  if (a.kv_ranges > 1)
+    for (int c = 0; c <= a.kv_ranges; ++c) a.kvb[c] = kv_bounds[c];
+  a.Bseq = B * a.kv_ranges;
+  a.nchunks = static_cast<int>(ceil_div64(max_len, kSmoothChunk));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (a.nchunks > 0) {
-    dim3 grid(a.nchunks, B, Hkv);
+    dim3 grid(a.nchunks, a.Bseq, Hkv);
     if (dt == SKV_BF16) kmean_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
     else kmean_partial_kernel<__half><<<grid, 256, 0, st>>>(a);
   }
   // the mean itself is needed here only to materialise K'; otherwise the
   // prefill kernel adds up the per-chunk partial sums of its own KV range
-  if (k_smoothed != nullptr) kmean_finalize_kernel<<<B * Hkv, D, 0, st>>>(a);
+  if (k_smoothed != nullptr) kmean_finalize_kernel<<<a.Bseq * Hkv, D, 0, st>>>(a);
   if (k_smoothed != nullptr && a.nchunks > 0) {
-    dim3 grid(a.nchunks, B, Hkv);
+    dim3 grid(a.nchunks, a.Bseq, Hkv);
     if (dt == SKV_BF16) ksmooth_write_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
     else ksmooth_write_kernel<__half><<<grid, 256, 0, st>>>(a);
   }

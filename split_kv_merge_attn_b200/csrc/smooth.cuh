@@ -15,26 +15,35 @@ namespace skv {
 
 constexpr int kSmoothChunk = 256;
 
+// A "range" is the key range one mean is taken over: a batch entry (dense), a
+// varlen sequence, or, in a multi-chunk dense call, KV chunk c of batch entry
+// b (range index b * nranges_per_batch + c, keys [kvb[c], kvb[c+1])).
 struct SmoothArgs {
   const void* k;
   void* k_out;          // K' (materialising mode) or null
   float* partial;       // [nchunks, Bseq, Hkv, D]
   float* kmean;         // [Bseq, Hkv, D]
   const int* cu_k;      // varlen offsets or null
-  int Bseq, Hkv, Sk, D;
-  int nchunks;
+  int Bseq, Hkv, Sk, D; // Bseq: number of ranges
+  int nchunks;          // 256-key chunks of the longest range
   int layout;           // 0 HND, 1 NHD, 2 TND
+  int kv_ranges;        // dense: key ranges per batch entry (1 = all Sk keys)
+  int kvb[kMaxKvChunks + 1];
 };
 
-// element offset of key s (inside its batch / sequence) of kv head hkv
-__device__ __forceinline__ int64_t smooth_row_off(const SmoothArgs& a, int b, int hkv, int s) {
-  if (a.layout == 0) return ((static_cast<int64_t>(b) * a.Hkv + hkv) * a.Sk + s) * a.D;
-  if (a.layout == 1) return ((static_cast<int64_t>(b) * a.Sk + s) * a.Hkv + hkv) * a.D;
-  return (static_cast<int64_t>(a.cu_k[b] + s) * a.Hkv + hkv) * a.D;
+// element offset of key s (inside its range) of kv head hkv
+__device__ __forceinline__ int64_t smooth_row_off(const SmoothArgs& a, int r, int hkv, int s) {
+  if (a.layout == 2) return (static_cast<int64_t>(a.cu_k[r] + s) * a.Hkv + hkv) * a.D;
+  const int b = r / a.kv_ranges;
+  const int key = a.kvb[r - b * a.kv_ranges] + s;
+  if (a.layout == 0) return ((static_cast<int64_t>(b) * a.Hkv + hkv) * a.Sk + key) * a.D;
+  return ((static_cast<int64_t>(b) * a.Sk + key) * a.Hkv + hkv) * a.D;
 }
 
-__device__ __forceinline__ int smooth_len(const SmoothArgs& a, int b) {
-  return a.layout == 2 ? a.cu_k[b + 1] - a.cu_k[b] : a.Sk;
+__device__ __forceinline__ int smooth_len(const SmoothArgs& a, int r) {
+  if (a.layout == 2) return a.cu_k[r + 1] - a.cu_k[r];
+  const int c = r % a.kv_ranges;
+  return a.kvb[c + 1] - a.kvb[c];
 }
 
 // grid (nchunks, Bseq, Hkv), 256 threads: (D/8) column vectors x (256/(D/8)) row lanes.

@@ -321,6 +321,36 @@ def test_chunked_merge_equals_full_with_smoothing():
         assert np.abs(om_bad - o).max() > 1e-4
 
 
+def test_chunked_partials_against_torch_float64():
+    """oracle.chunked: each part is PyTorch float64 attention over that chunk's
+    keys alone (an empty chunk gives O = 0, LSE = -inf), in HND and NHD, and the
+    merge of the parts is PyTorch float64 attention over all keys."""
+    d = W.dense_case(2, 4, 2, 7, 45, 8, seed=21, q_mult=3.0)
+    bounds = [0, 9, 9, 30, 45]
+    q, k, v = (d[x].double() for x in "qkv")
+    kr, vr = k.repeat_interleave(2, dim=1), v.repeat_interleave(2, dim=1)
+    for layout in ("HND", "NHD"):
+        args = [W.to_layout(d[x], layout) for x in "qkv"]
+        o_p, l_p = O.chunked(*args, d["scale"], bounds, layout=layout)
+        assert o_p.shape[0] == 4 and l_p.shape == (4, 2, 4, 7)
+        for c in range(4):
+            a, e = bounds[c], bounds[c + 1]
+            if a == e:
+                assert np.all(o_p[c] == 0) and np.all(np.isneginf(l_p[c]))
+                continue
+            s = torch.einsum("bhid,bhjd->bhij", q, kr[:, :, a:e]) * d["scale"]
+            o_t = torch.softmax(s, -1) @ vr[:, :, a:e]
+            l_t = torch.logsumexp(s, -1) / math.log(2)
+            o_c = o_p[c] if layout == "HND" else o_p[c].transpose(0, 2, 1, 3)
+            np.testing.assert_allclose(o_c, o_t.numpy(), atol=1e-12)
+            np.testing.assert_allclose(l_p[c], l_t.numpy(), atol=1e-12)
+    o_p, l_p = O.chunked(d["q"], d["k"], d["v"], d["scale"], bounds)
+    om, lm = O.merge(o_p, l_p)
+    s = torch.einsum("bhid,bhjd->bhij", q, kr) * d["scale"]
+    np.testing.assert_allclose(om, (torch.softmax(s, -1) @ vr).numpy(), atol=1e-12)
+    np.testing.assert_allclose(lm, (torch.logsumexp(s, -1) / math.log(2)).numpy(), atol=1e-12)
+
+
 # ------------------------------------------------------- varlen and decode
 
 def test_varlen_equals_dense_per_sequence():
