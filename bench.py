@@ -4,8 +4,9 @@
 One step = one pass over every operation of the path at the workloads' full
 sizes, inputs resident in HBM:
   * varlen TND prefill, H=24, D=128, seqlens {512,1024,2048,4096}   (attn_fwd_lse)
-  * ring-style chunked prefill, B=1, H=16, S_q=4096, S_k=16384, D=128: four
-    KV chunks of 4096 with smooth_k, then merge_state of the four partials
+  * ring-style chunked prefill, B=1, H=16, S_q=4096, S_k=16384, D=128: the
+    partials of four KV chunks of 4096, each smoothed by its own mean, in one
+    attn_fwd_lse_chunks launch, then merge_state of the four partials
   * split-KV decode D=128 (H_q=32, H_kv=8) and D=256 (H_q=16, H_kv=4),
     Lkv=32768, Lq in {1, 4}                                      (attn_splitkv_decode)
 The headline value is prefill-dominated TFLOP/s (algorithmic FLOPs of the
@@ -191,8 +192,7 @@ def run_ours(args, rank, world, dist):
     cuq4, cuk4 = c4["cu_seqlens_q"].to(dev), c4["cu_seqlens_k"].to(dev)
     q5 = c5["q"].to(dev)
     b5 = c5["chunk_bounds"]
-    k5 = [c5["k"][:, :, a:e].contiguous().to(dev) for a, e in zip(b5[:-1], b5[1:])]
-    v5 = [c5["v"][:, :, a:e].contiguous().to(dev) for a, e in zip(b5[:-1], b5[1:])]
+    k5, v5 = c5["k"].to(dev), c5["v"].to(dev)   # the whole key range; the chunks are bounds into it
     dec_in = []
     for (name, Hq, Hkv, D, Lq, Lkv) in DECODE_SHAPES:
         if D == 128:
@@ -210,8 +210,8 @@ def run_ours(args, rank, world, dist):
                       dtype=torch.uint8, device=dev)
     o5p = torch.empty((4,) + tuple(q5.shape), dtype=q5.dtype, device=dev)
     l5p = torch.empty(4, 1, 16, 4096, dtype=torch.float32, device=dev)
-    ws5 = torch.empty(skv.attn_fwd_lse_workspace(1, 16, 16, 4096, 128, "bf16", "HND", 1), dtype=torch.uint8,
-                      device=dev)
+    ws5 = torch.empty(skv.attn_fwd_lse_chunks_workspace(1, 16, 16, 16384, 128, 4, "bf16", "HND", 1),
+                      dtype=torch.uint8, device=dev)
     out5 = torch.empty_like(q5)
     lse5 = torch.empty(1, 16, 4096, dtype=torch.float32, device=dev)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -236,9 +236,8 @@ def run_ours(args, rank, world, dist):
                          max_seqlen_q=4096, max_seqlen_k=4096, out=out4, lse=lse4, workspace=ws4)
 
     def call_cfg5():
-        for c in range(4):
-            skv.attn_fwd_lse(q5, k5[c], v5[c], scale, layout="HND", smooth_k=1, out=o5p[c], lse=l5p[c],
-                             workspace=ws5)
+        # the four chunks' partials (each smoothed by its own mean) in one launch, then their merge
+        skv.attn_fwd_lse_chunks(q5, k5, v5, b5, scale, layout="HND", smooth_k=1, out=o5p, lse=l5p, workspace=ws5)
         skv.merge_state(o5p, l5p, "HND", out=out5, lse=lse5)
 
     def call_decode(i):
@@ -320,7 +319,10 @@ def run_ours(args, rank, world, dist):
         FLOPS_CFG5 / (detail["cfg5_chunked_prefill_merge"]["us_in_step"] * 1e-6) / 1e12, 1)
     detail["cfg4_varlen_prefill"]["tflops"] = round(pf_tflops, 1)
 
-    def time_graph(fn, reps):
+    def time_graph(fn, reps, per_replay=1, flush=True):
+        """Mean of the middle 60% of `reps` graph replays of fn (captured once),
+        divided by `per_replay` (the calls one replay makes); L2 flushed before
+        each replay unless the replay's own inputs exceed it."""
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
@@ -334,13 +336,14 @@ def run_ours(args, rank, world, dist):
         torch.cuda.synchronize()
         ts = []
         for _ in range(reps):
-            flush_l2()
+            if flush:
+                flush_l2()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             g.replay()
             e1.record()
             torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1) * 1e3)
+            ts.append(e0.elapsed_time(e1) * 1e3 / per_replay)
         ts.sort()
         del g
         # mean of the middle 60%: event times come in ~2 us ticks here, so a
@@ -348,15 +351,40 @@ def run_ours(args, rank, world, dist):
         k = len(ts) // 5
         return sum(ts[k:len(ts) - k]) / (len(ts) - 2 * k)
 
+    # The fixed cost of one isolated replay (graph launch, one tiny kernel,
+    # events): a floor under every "graph_us" below.
+    tiny = torch.zeros(1, device=dev)
+    floor_us = time_graph(lambda: tiny.add_(1.0), 50)
+    detail["graph_floor_us"] = {"graph_us": round(floor_us, 2),
+                                "what": "one graph replay of a one-element kernel, timed like the operators below"}
+    N_B2B = 6
+
+    def back_to_back(make_call, sets):
+        """Per-call time of N_B2B calls replayed in one graph, call i on input
+        set i: the sets together exceed L2, so each call reads its inputs from
+        HBM, and the launch cost of one call overlaps the previous call."""
+        calls = [make_call(x) for x in sets]
+
+        def run():
+            for c in calls:
+                c()
+        return time_graph(run, 20, per_replay=len(calls), flush=False)
+
     for i, (name, Hq, Hkv, D, Lq, Lkv) in enumerate(DECODE_SHAPES):
         us = time_graph(lambda i=i: call_decode(i), 50)
         gbs = decode_kv_bytes(Hkv, D, Lkv) / (us * 1e-6) / 1e9
-        detail[name].update({"graph_us": round(us, 2), "kv_gbs": round(gbs, 1),
-                             "hbm_frac": round(gbs / peaks["hbm_gbs"], 3), "splits": dec_buf[i][3],
-                             "pages_a100_us": PAGES_A100_US.get(("decode", D, Lq, Lkv))})
-        # the single-launch variant (in-kernel merge by the last CTA of each group)
         _, q, k, v, sc = dec_in[i]
         o, l, ws, splits = dec_buf[i]
+        kv_sets = [(k, v)] + [(k.clone(), v.clone()) for _ in range(N_B2B - 1)]
+        us_b = back_to_back(lambda kv: (lambda: skv.attn_splitkv_decode(q, kv[0], kv[1], sc, num_splits=splits, out=o,
+                                                                        lse=l, workspace=ws)), kv_sets)
+        del kv_sets
+        gbs_b = decode_kv_bytes(Hkv, D, Lkv) / (us_b * 1e-6) / 1e9
+        detail[name].update({"graph_us": round(us, 2), "kv_gbs": round(gbs, 1),
+                             "b2b_us": round(us_b, 2), "b2b_kv_gbs": round(gbs_b, 1),
+                             "hbm_frac": round(gbs_b / peaks["hbm_gbs"], 3), "splits": dec_buf[i][3],
+                             "pages_a100_us": PAGES_A100_US.get(("decode", D, Lq, Lkv))})
+        # the single-launch variant (in-kernel merge by the last CTA of each group)
         wsz = torch.zeros_like(ws)
         us_f = time_graph(lambda: skv.attn_splitkv_decode(q, k, v, sc, num_splits=splits, out=o, lse=l,
                                                           workspace=wsz, fused=True), 50)
@@ -375,25 +403,55 @@ def run_ours(args, rank, world, dist):
         o, l = torch.empty_like(q), torch.empty(B, Hq, Lq, dtype=torch.float32, device=dev)
         us = time_graph(lambda: skv.attn_splitkv_decode(q, k, v, sc, num_splits=splits, out=o, lse=l, workspace=ws), 50)
         gbs = decode_kv_bytes(Hkv, D, Lkv) / (us * 1e-6) / 1e9
+        n_sets = max(N_B2B, -(-8 * 126 * 2 ** 20 // decode_kv_bytes(Hkv, D, Lkv)))  # >= 8 L2 sizes in all
+        kv_sets = [(k, v)] + [(k.clone(), v.clone()) for _ in range(n_sets - 1)]
+        us_b = back_to_back(lambda kv: (lambda: skv.attn_splitkv_decode(q, kv[0], kv[1], sc, num_splits=splits, out=o,
+                                                                        lse=l, workspace=ws)), kv_sets)
+        del kv_sets
+        gbs_b = decode_kv_bytes(Hkv, D, Lkv) / (us_b * 1e-6) / 1e9
         detail[f"decode_d{D}_lq{Lq}_lkv{Lkv}"] = {"graph_us": round(us, 2), "kv_gbs": round(gbs, 1),
-                                                  "hbm_frac": round(gbs / peaks["hbm_gbs"], 3), "splits": splits,
+                                                  "b2b_us": round(us_b, 2), "b2b_kv_gbs": round(gbs_b, 1),
+                                                  "hbm_frac": round(gbs_b / peaks["hbm_gbs"], 3), "splits": splits,
                                                   "pages_a100_us": a100}
         del q, k, v, o, l, ws
     # merge_state of workload 5 alone (HBM bound)
     us_m = time_graph(lambda: skv.merge_state(o5p, l5p, "HND", out=out5, lse=lse5), 50)
+    m_sets = [(o5p, l5p)] + [(o5p.clone(), l5p.clone()) for _ in range(N_B2B - 1)]
+    us_mb = back_to_back(lambda ol: (lambda: skv.merge_state(ol[0], ol[1], "HND", out=out5, lse=lse5)), m_sets)
+    del m_sets
     detail["merge_state_cfg5"] = {"graph_us": round(us_m, 2),
                                   "gbs": round(MERGE5_BYTES / (us_m * 1e-6) / 1e9, 1),
-                                  "hbm_frac": round(MERGE5_BYTES / (us_m * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)}
+                                  "b2b_us": round(us_mb, 2),
+                                  "b2b_gbs": round(MERGE5_BYTES / (us_mb * 1e-6) / 1e9, 1),
+                                  "hbm_frac": round(MERGE5_BYTES / (us_mb * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)}
+    # the same chunked workload as four separate attn_fwd_lse calls (context
+    # for the one-launch chunks call of the step)
+    k5c = [k5[:, :, a:e].contiguous() for a, e in zip(b5[:-1], b5[1:])]
+    v5c = [v5[:, :, a:e].contiguous() for a, e in zip(b5[:-1], b5[1:])]
+    ws5s = torch.empty(skv.attn_fwd_lse_workspace(1, 16, 16, 4096, 128, "bf16", "HND", 1), dtype=torch.uint8,
+                       device=dev)
+
+    def cfg5_four_calls():
+        for c in range(4):
+            skv.attn_fwd_lse(q5, k5c[c], v5c[c], scale, smooth_k=1, out=o5p[c], lse=l5p[c], workspace=ws5s)
+        skv.merge_state(o5p, l5p, "HND", out=out5, lse=lse5)
+    us_4 = time_graph(cfg5_four_calls, 20)
+    us_1 = time_graph(call_cfg5, 20)
+    detail["cfg5_chunked_prefill_merge"].update({
+        "graph_us": round(us_1, 2), "graph_tflops": round(FLOPS_CFG5 / (us_1 * 1e-6) / 1e12, 1),
+        "four_calls_graph_us": round(us_4, 2)})
+    del k5c, v5c
     # causal variants: prefill of the first workload-5 chunk with its own queries
     # (Sq = Sk = 4096) and the Lq = 4 decode of workload 2 at Lkv 32768
+    k5_0, v5_0 = k5[:, :, b5[0]:b5[1]].contiguous(), v5[:, :, b5[0]:b5[1]].contiguous()  # the first chunk
     oc = torch.empty_like(q5)
     lc = torch.empty(1, 16, 4096, dtype=torch.float32, device=dev)
-    us_c = time_graph(lambda: skv.attn_fwd_lse(q5, k5[0], v5[0], scale, out=oc, lse=lc, causal=True), 20)
+    us_c = time_graph(lambda: skv.attn_fwd_lse(q5, k5_0, v5_0, scale, out=oc, lse=lc, causal=True), 20)
     detail["causal_prefill_h16_s4096"] = {"graph_us": round(us_c, 2),
                                           "tflops": round(FLOPS_CAUSAL_CHUNK / (us_c * 1e-6) / 1e12, 1)}
     # INT8 Q K'^T with smooth_k on the same chunk (mean, codes and prefill: the whole call)
     ws8 = torch.empty(skv.attn_fwd_lse_int8_workspace(1, 16, 16, 4096, 4096), dtype=torch.uint8, device=dev)
-    us_8 = time_graph(lambda: skv.attn_fwd_lse_int8(q5, k5[0], v5[0], scale, out=oc, lse=lc, workspace=ws8), 20)
+    us_8 = time_graph(lambda: skv.attn_fwd_lse_int8(q5, k5_0, v5_0, scale, out=oc, lse=lc, workspace=ws8), 20)
     detail["int8_smooth_prefill_h16_s4096"] = {"graph_us": round(us_8, 2),
                                                "tflops": round(FLOPS_CFG5 / 4 / (us_8 * 1e-6) / 1e12, 1)}
     i4 = [n for n, *_r in DECODE_SHAPES].index("decode_d128_lq4_lkv32768")
@@ -418,13 +476,15 @@ def run_ours(args, rank, world, dist):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded randn, workloads/)",
             "config": {"workload": "one pass over: varlen TND prefill (H24 D128 seqlens 512..4096) + chunked "
-                                   "ring-style prefill with smooth_k (B1 H16 Sq4096 Sk16384 D128, 4 chunks) + "
+                                   "ring-style prefill with smooth_k (B1 H16 Sq4096 Sk16384 D128, 4 chunks in one launch) + "
                                    "merge_state + split-KV decode (D128 Hq32/Hkv8 and D256 Hq16/Hkv4, Lkv 32768, "
                                    "Lq 1 and 4)",
                        "algorithmic_gflop_per_step": round(step_flops / 1e9, 2),
                        "l2": "flushed (256 MB write + 256 MB read) before every timed step and replay",
-                       "detail_timing": "decode and merge_state alone: CUDA-graph replays, mean of the middle 60% "
-                                        "of 50 (L2 flushed before each)",
+                       "detail_timing": "decode and merge_state alone: graph_us = one CUDA-graph replay (L2 flushed "
+                                        "before each; mean of the middle 60% of 50; it includes the fixed cost in "
+                                        "graph_floor_us); b2b_us = per-call time of back-to-back calls in one graph "
+                                        "over input sets larger than L2 together; hbm_frac uses b2b_us",
                        "parallelism": f"replicas x{world} (independent work per GPU, no exchange)"},
             "roofline": roofline, "detail": detail, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clocks, "cpu_baseline": cpu, "peaks": peaks,
@@ -441,11 +501,10 @@ def run_e2e(args, dev, host, skv, torch, step_flops, world, dist):
     hcu = pin(c4["cu_seqlens_q"])
     hq5 = pin(c5["q"])
     b5 = c5["chunk_bounds"]
-    hk5 = [pin(c5["k"][:, :, a:e].contiguous()) for a, e in zip(b5[:-1], b5[1:])]
-    hv5 = [pin(c5["v"][:, :, a:e].contiguous()) for a, e in zip(b5[:-1], b5[1:])]
+    hk5, hv5 = pin(c5["k"]), pin(c5["v"])
     hdec = [(pin(host[n]["q"]), pin(host[n]["k"]), pin(host[n]["v"]), host[n]["scale"]) for (n, *_r) in DECODE_SHAPES]
     sc = D128 ** -0.5
-    h2d = sum(t.numel() * t.element_size() for t in [hq4, hk4, hv4, hcu, hcu, hq5] + hk5 + hv5)
+    h2d = sum(t.numel() * t.element_size() for t in [hq4, hk4, hv4, hcu, hcu, hq5, hk5, hv5])
     h2d += sum(q.numel() * q.element_size() + k.numel() * k.element_size() * 2 for q, k, v, s in hdec)
     # outputs read back: O (bf16) and LSE (fp32) of every call
     d2h_o = [torch.empty_like(hq4, device="cpu").pin_memory(), torch.empty(24, hq4.shape[0]).pin_memory(),
@@ -460,9 +519,9 @@ def run_e2e(args, dev, host, skv, torch, step_flops, world, dist):
         o4, l4 = skv.attn_fwd_lse(q4, k4, v4, sc, layout="TND", cu_seqlens_q=cu, cu_seqlens_k=cu, max_seqlen_q=4096,
                                   max_seqlen_k=4096)
         q5 = hq5.to(dev, non_blocking=True)
-        parts = [skv.attn_fwd_lse(q5, k.to(dev, non_blocking=True), v.to(dev, non_blocking=True), sc, smooth_k=1)
-                 for k, v in zip(hk5, hv5)]
-        o5, l5 = skv.merge_state(torch.stack([p[0] for p in parts]), torch.stack([p[1] for p in parts]))
+        op5, lp5 = skv.attn_fwd_lse_chunks(q5, hk5.to(dev, non_blocking=True), hv5.to(dev, non_blocking=True), b5,
+                                           sc, smooth_k=1)
+        o5, l5 = skv.merge_state(op5, lp5)
         outs = [o4, l4, o5, l5]
         dec_o, dec_l = [], []
         for q, k, v, s in hdec:
@@ -588,6 +647,93 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- ring (context parallel)
+
+RING_METRIC = "ring attention fwd+LSE TFLOP/s (context-parallel, KV shards passed rank to rank)"
+
+
+def ring_job(dist, rank: int, world: int, device, steps: int, warmup: int, shard: int = 4096, H: int = 16,
+             D: int = 128, seed: int = 0, dtype=None, attn=None, merge=None, exchange=None):
+    """Context-parallel (ring) attention timed as a job: one sequence of
+    shard * world tokens, rank r holding tokens [r*shard, (r+1)*shard) of q, k
+    and v ([1, H, shard, D]).  Each step every rank computes the attention of
+    its queries over all keys with split_kv_merge_attn_b200.ring (one partial
+    per hop while the next key/value shard travels, then merge_state).  At
+    world = 4 and shard = 4096 every rank does the work of the chunked
+    workload (4096 queries over 16384 keys in four chunks).  Returns the
+    job's numbers and this rank's last (O, LSE).  attn / merge / exchange
+    replace the library's kernels and the point-to-point exchange (the CPU
+    tests use that to run this function on gloo ranks)."""
+    import torch
+    from split_kv_merge_attn_b200.ring import ring_attn_fwd_lse
+    dtype = dtype or torch.bfloat16
+    g = torch.Generator().manual_seed(seed * 1000 + rank)   # this rank's shard of the sequence
+    q = torch.randn(1, H, shard, D, generator=g).to(dtype).to(device)
+    k = torch.randn(1, H, shard, D, generator=g).to(dtype).to(device)
+    v = torch.randn(1, H, shard, D, generator=g).to(dtype).to(device)
+    scale = D ** -0.5
+    cuda = torch.device(device).type == "cuda"
+
+    def step():
+        return ring_attn_fwd_lse(q, k, v, scale, attn=attn, merge=merge, exchange=exchange)
+
+    res = None
+    for _ in range(warmup):
+        res = step()
+    if cuda:
+        torch.cuda.synchronize()
+    dist.barrier()
+    if cuda:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        res = step()
+    if cuda:
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+    else:
+        ms = (time.perf_counter() - t0) * 1e3 / steps
+    dist.barrier()
+    ms = max_over_ranks(ms, dist if world > 1 else None, device)
+    flops_rank = attn_flops(H * shard * shard * world, D)
+    return {"ms": ms, "value": job_value(flops_rank, world, ms), "flops_per_rank": flops_rank,
+            "result": res, "inputs": (q, k, v, scale)}
+
+
+def run_ring(args, rank, world, dist):
+    import torch
+    import split_kv_merge_attn_b200 as skv
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if dist is None:  # one rank: a trivial group so the ring code runs its one hop
+        import datetime
+        import torch.distributed as tdist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29511")
+        tdist.init_process_group("gloo", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60))
+        dist = tdist
+    launches0 = skv.launch_count()
+    r = ring_job(dist, rank, world, dev, args.steps, args.warmup)
+    launches = skv.launch_count() - launches0
+    assert skv.device_error() == 0
+    if rank == 0:
+        line = {"metric": RING_METRIC, "value": round(r["value"], 2), "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms"], 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded randn per rank)",
+                "config": {"workload": f"ring attention over one sequence of {4096 * world} tokens, 4096 per rank, "
+                                       "H16 D128, non-causal; per hop one attn_fwd_lse partial while the next "
+                                       "K/V shard travels (torch.distributed P2P: NCCL on GPUs), then merge_state",
+                           "parallelism": f"context-parallel ring x{world}",
+                           "l2": "not flushed (each hop's shard is new data on the rank)"},
+                "gpu_launches": int(launches)}
+        print(json.dumps(line), flush=True)
+    if world == 1:
+        dist.destroy_process_group()
+
+
 # ---------------------------------------------------------------- main
 
 def run_case(args):
@@ -637,6 +783,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None, help="run one operation only (for profiler captures)")
+    ap.add_argument("--ring", action="store_true", help="time context-parallel ring attention across the ranks")
     args = ap.parse_args()
     if args.case:
         run_case(args)
@@ -650,6 +797,9 @@ def main():
         return
     dist = init_distributed(world, "nccl")
     try:
+        if args.ring:
+            run_ring(args, rank, world, dist)
+            return
         run_ours(args, rank, world, dist)
     finally:
         if dist is not None:

@@ -41,17 +41,79 @@ constexpr int kPfBN = 128;          // keys per KV tile
 constexpr int kPfThreads = 320;
 constexpr float kPfRescaleThreshold = 8.0f;
 
+// Tuning switches (compile time) of the softmax's exponent pass, which is
+// bound by the special-function unit (ex2 and the packing conversion share it):
+//   SKV_PF_POLY_PAIRS  of every 16 pairs of probabilities, this many are
+//                      computed on the FMA pipe (poly_exp2_pair) instead of ex2;
+//   SKV_PF_INT_PACK    1: round the probabilities to 16 bits with integer
+//                      operations instead of the conversion instruction.
+#ifndef SKV_PF_POLY_PAIRS
+#define SKV_PF_POLY_PAIRS 0
+#endif
+#ifndef SKV_PF_INT_PACK
+#define SKV_PF_INT_PACK 0
+#endif
+
+// 2^x on the FMA pipe for x in [-126, 2^22): x = n + f with n = round(x) (the
+// 1.5 * 2^23 addition) and f in [-1/2, 1/2]; 2^f by the degree-3 polynomial
+// of least maximum relative error on [-1/2, 1/2] (7.5e-5; the coefficients
+// are those printed by exp2_poly_fit.py in this directory, a Remez exchange);
+// 2^n is an addition to the exponent field.  Arguments below -126 are clamped
+// there (results < 2^-125).
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+
+__device__ __forceinline__ void poly_exp2_pair(uint64_t x2, float& p0, float& p1) {
+  float2 x = f2_unpack(x2);
+  const uint64_t xc = f2_pack(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
+  const uint64_t y = fadd2(xc, f2_pack(12582912.f, 12582912.f));    // round(x) in the low mantissa bits
+  const uint64_t n = fadd2(y, f2_pack(-12582912.f, -12582912.f));   // round(x) as a float
+  const uint64_t f = ffma2(n, f2_pack(-1.f, -1.f), xc);              // x - round(x), exact
+  uint64_t q = ffma2(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  q = ffma2(q, f, f2_pack(kExp2C1, kExp2C1));
+  q = ffma2(q, f, f2_pack(kExp2C0, kExp2C0));
+  const float2 qf = f2_unpack(q), yf = f2_unpack(y);
+  p0 = __uint_as_float(__float_as_uint(qf.x) + (__float_as_uint(yf.x) << 23));
+  p1 = __uint_as_float(__float_as_uint(qf.y) + (__float_as_uint(yf.y) << 23));
+}
+
+// Two non-negative finite floats rounded to nearest-even 16-bit pairs with
+// integer operations (bf16: the upper half after adding 0x7FFF plus the lowest
+// kept bit; fp16 goes through the conversion instruction).
+template <typename T>
+__device__ __forceinline__ uint32_t pack2_p(float lo, float hi) {
+  if constexpr (SKV_PF_INT_PACK && std::is_same<T, __nv_bfloat16>::value) {
+    uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+    a += 0x7FFFu + ((a >> 16) & 1u);
+    b += 0x7FFFu + ((b >> 16) & 1u);
+    return __byte_perm(a, b, 0x7632);
+  } else {
+    return pack2<T>(lo, hi);
+  }
+}
+
 // Exponentiates 64 logits (32 pairs) of one row: p = 2^(s * scale_log2 + nb),
 // packs them as 16-bit pairs and accumulates the row sum in packed fp32 pairs.
-template <typename T>
+// kPoly: a tile without masked keys, where SKV_PF_POLY_PAIRS of every 16 pairs
+// go to the FMA pipe (a masked key must give exactly 0, which ex2 does).
+template <bool kPoly, typename T>
 __device__ __forceinline__ void exp_pack_64(const float (&sv)[64], uint64_t sc2, uint64_t nb2, uint32_t (&pk)[32],
                                             uint64_t (&ps2)[2]) {
 #pragma unroll
   for (int e = 0; e < 32; ++e) {
-    const float2 x = f2_unpack(ffma2(f2_pack(sv[2 * e], sv[2 * e + 1]), sc2, nb2));
-    const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+    const uint64_t x2 = ffma2(f2_pack(sv[2 * e], sv[2 * e + 1]), sc2, nb2);
+    float p0, p1;
+    if (kPoly && ((e % 16) * SKV_PF_POLY_PAIRS) % 16 < SKV_PF_POLY_PAIRS) {
+      poly_exp2_pair(x2, p0, p1);
+    } else {
+      const float2 x = f2_unpack(x2);
+      p0 = ex2_approx(x.x);
+      p1 = ex2_approx(x.y);
+    }
     ps2[e & 1] = fadd2(ps2[e & 1], f2_pack(p0, p1));
-    pk[e] = pack2<T>(p0, p1);
+    pk[e] = pack2_p<T>(p0, p1);
   }
 }
 
@@ -317,49 +379,60 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // phases alternate on the exp units):
     //   S_0(0) S_1(0) PV_0(0) | S_0(j) PV_1(j-1) S_1(j) PV_0(j) | PV_1(last)
     // S_t(j) overwrites the TMEM columns that PV_t(j-1) reads P_t from; the two
-    // are issued back to back by this one thread and executed in issue order,
-    // the ordering NVIDIA's CUTLASS Blackwell FMHA also relies on.
-    if (lane == 0) {
+    // are issued back to back by one thread and executed in issue order, the
+    // ordering NVIDIA's CUTLASS Blackwell FMHA also relies on.
+    // The whole warp runs this role in step (waits, descriptor arithmetic),
+    // and one elected lane issues each group of MMAs and every commit: the
+    // operands stay warp-uniform, so they need no per-MMA move from a
+    // thread's registers into the uniform ones tcgen05.mma reads.
+    {
       const uint32_t ring_addr = smem_u32(ring);
       const uint32_t q0 = smem_u32(qtile[0]), q1 = smem_u32(qtile[1]);
       const uint32_t s0c = tmem + Cfg::kSCol0, s1c = tmem + Cfg::kSCol1;
       const uint32_t o0c = tmem + Cfg::kOCol0, o1c = tmem + Cfg::kOCol1;
       // Shared-memory descriptors are built once; every MMA then only adds a
       // constant to the start-address field (shared addresses are < 256 KB, so
-      // the 14-bit field never carries).  This keeps the issuing thread cheap:
-      // it shares its scheduler with two softmax warps.
+      // the 14-bit field never carries).
       const uint64_t dq0 = tc5::smem_desc(q0, 16, 1024), dq1 = tc5::smem_desc(q1, 16, 1024);
       const uint64_t dk_base = tc5::smem_desc(ring_addr, 16, 1024);
       const uint64_t dv_base = tc5::smem_desc(ring_addr, Cfg::kBoxBytes, 1024);
       auto issue_s = [&](uint64_t dq, uint32_t sc, int u) {
         const uint64_t dk = dk_base + static_cast<uint64_t>(((u % Cfg::kStages) * Cfg::kKVTileBytes) >> 4);
-        // one MMA per 32 bytes of a Q/K row (K = 16 for 16-bit, 32 for int8)
+        if (elect_one()) {
+          // one MMA per 32 bytes of a Q/K row (K = 16 for 16-bit, 32 for int8)
 #pragma unroll
-        for (int kk = 0; kk < (kI8 ? D / 32 : D / 16); ++kk) {
-          const uint64_t o = static_cast<uint64_t>(((kk >> 2) * Cfg::kBoxBytes + (kk & 3) * 32) >> 4);
-          if constexpr (kI8) tc5::mma_ss_i8(sc, dq + o, dk + o, kIdescQK, kk > 0 ? 1u : 0u);
-          else tc5::mma_ss(sc, dq + o, dk + o, kIdescQK, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < (kI8 ? D / 32 : D / 16); ++kk) {
+            const uint64_t o = static_cast<uint64_t>(((kk >> 2) * Cfg::kBoxBytes + (kk & 3) * 32) >> 4);
+            if constexpr (kI8) tc5::mma_ss_i8(sc, dq + o, dk + o, kIdescQK, kk > 0 ? 1u : 0u);
+            else tc5::mma_ss(sc, dq + o, dk + o, kIdescQK, kk > 0 ? 1u : 0u);
+          }
         }
+        __syncwarp();
       };
       auto issue_pv_half = [&](uint32_t sc, uint32_t oc, int u, bool acc, int hf) {
         const uint64_t dv = dv_base + static_cast<uint64_t>(((u % Cfg::kStages) * Cfg::kKVTileBytes) >> 4);
+        if (elect_one()) {
 #pragma unroll
-        for (int k4 = 0; k4 < kPfBN / 32; ++k4) {
-          const int kk = hf * (kPfBN / 32) + k4;
-          tc5::mma_ts(oc, sc + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
-                      (acc || kk > 0) ? 1u : 0u);
+          for (int k4 = 0; k4 < kPfBN / 32; ++k4) {
+            const int kk = hf * (kPfBN / 32) + k4;
+            tc5::mma_ts(oc, sc + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
+                        (acc || kk > 0) ? 1u : 0u);
+          }
         }
+        __syncwarp();
       };
-      auto wait_kv = [&](int u) -> bool {
-        const bool r = mbar_wait(&kv_full[u % Cfg::kStages], (u / Cfg::kStages) & 1, abort_flag, kErrPrefillWait);
+      auto commit = [&](uint64_t* bar) {
+        if (elect_one()) tc5::commit(smem_u32(bar));
+        __syncwarp();
+      };
+      // every lane waits; the warp proceeds only on a common verdict
+      auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
+        const bool r = __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kErrPrefillWait));
         tc5::fence_after();
         return r;
       };
-      auto wait_p = [&](int t, int hf, int j) -> bool {
-        const bool r = mbar_wait(&p_half[2 * t + hf], j & 1, abort_flag, kErrPrefillWait);
-        tc5::fence_after();
-        return r;
-      };
+      auto wait_kv = [&](int u) -> bool { return wait_bar(&kv_full[u % Cfg::kStages], (u / Cfg::kStages) & 1); };
+      auto wait_p = [&](int t, int hf, int j) -> bool { return wait_bar(&p_half[2 * t + hf], j & 1); };
       // PV of tile t for KV tile j, started on the first 64 keys of P while the
       // softmax still exponentiates the second 64
       auto issue_pv = [&](int t, int u, bool acc, int j) -> bool {
@@ -370,40 +443,40 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         issue_pv_half(sc, oc, u, acc, 1);
         return true;
       };
-      auto release = [&](int u) { tc5::commit(smem_u32(&kv_empty[u % Cfg::kStages])); };
+      auto release = [&](int u) { commit(&kv_empty[u % Cfg::kStages]); };
       const bool two = nt == 2;
 
-      bool ok = mbar_wait(q_full, 0, abort_flag, kErrPrefillWait) && wait_kv(0);
+      bool ok = wait_bar(q_full, 0) && wait_kv(0);
       if (ok) {
         issue_s(dq0, s0c, 0);
-        tc5::commit(smem_u32(&s_full[0]));
+        commit(&s_full[0]);
         if (two) {
           issue_s(dq1, s1c, 0);
-          tc5::commit(smem_u32(&s_full[1]));
+          commit(&s_full[1]);
         }
         release(0);
         ok = wait_kv(1) && issue_pv(0, 1, false, 0);
-        if (ok && nkv == 1) tc5::commit(smem_u32(&o_full[0]));
+        if (ok && nkv == 1) commit(&o_full[0]);
       }
       for (int j = 1; j < nkv && ok; ++j) {
         const int uk = 2 * j, uv = 2 * j + 1;
         if (!wait_kv(uk)) { ok = false; break; }
         issue_s(dq0, s0c, uk);
-        tc5::commit(smem_u32(&s_full[0]));
+        commit(&s_full[0]);
         if (two && !issue_pv(1, uv - 2, j - 1 > 0, j - 1)) { ok = false; break; }
         release(uv - 2);              // V_{j-1}: both of its PV products are issued
         if (two) {
           issue_s(dq1, s1c, uk);
-          tc5::commit(smem_u32(&s_full[1]));
+          commit(&s_full[1]);
         }
         release(uk);                  // K_j: both S products are issued
         if (!wait_kv(uv)) { ok = false; break; }
         if (!issue_pv(0, uv, true, j)) { ok = false; break; }
-        if (j == nkv - 1) tc5::commit(smem_u32(&o_full[0]));
+        if (j == nkv - 1) commit(&o_full[0]);
       }
-      if (ok && two && issue_pv(1, 2 * nkv - 1, nkv - 1 > 0, nkv - 1)) tc5::commit(smem_u32(&o_full[1]));
-      // every MMA this thread issued has completed before TMEM is released
-      tc5::commit(smem_u32(drain));
+      if (ok && two && issue_pv(1, 2 * nkv - 1, nkv - 1 > 0, nkv - 1)) commit(&o_full[1]);
+      // every MMA the elected lane issued has completed before TMEM is released
+      commit(drain);
       mbar_drain(drain, 0, 20000000ull);
     }
   } else {
@@ -561,7 +634,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (hf * 64 + c >= n_valid) sh[c] = -INFINITY;
           }
           uint32_t pk[32];
-          exp_pack_64<T>(sh, sc2, nb2, pk, ps2);
+          if (full_tile) exp_pack_64<true, T>(sh, sc2, nb2, pk, ps2);
+          else exp_pack_64<false, T>(sh, sc2, nb2, pk, ps2);
           tc5::st16(s_addr + hf * 32, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
           tc5::st16(s_addr + hf * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
           tc5::wait_st();

@@ -97,6 +97,18 @@ __device__ __forceinline__ float2 unpack2<__half>(uint32_t v) {
   return __half22float2(h);
 }
 
+// One lane of a converged warp (elect.sync over the full warp): the same lane
+// every time the whole warp executes it.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------- errors
 
 // Device error word (one per device).  Written with atomicCAS so the first
