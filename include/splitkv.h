@@ -40,7 +40,7 @@
  * argument on the host first and launch nothing if validation fails.
  *
  * Element types: bf16 or fp16 for q/k/v/out (q, k, v and out share one type);
- * LSE is always fp32.  Head dimension D in {64, 128, 256} (prefill: {64, 128}).
+ * LSE is always fp32.  Head dimension D in {64, 128, 256} (INT8 prefill: 128).
  * Pointers passed as tensors must be 16-byte aligned.
  *
  * Thread safety: entry points may be called from several host threads; calls
@@ -62,7 +62,7 @@ typedef struct CUstream_st* skv_stream_t;
 typedef enum {
   SKV_OK = 0,
   SKV_ERR_INVALID_ARG = 1,        /* a size, pointer, alignment or layout is invalid */
-  SKV_ERR_UNSUPPORTED = 2,        /* valid but not implemented (e.g. prefill D=256) */
+  SKV_ERR_UNSUPPORTED = 2,        /* valid but not implemented (e.g. D=96, fp32 inputs) */
   SKV_ERR_WORKSPACE_TOO_SMALL = 3,/* workspace_bytes < the *_workspace() query */
   SKV_ERR_CUDA = 4                /* a CUDA runtime/driver call failed; see skv_last_cuda_error */
 } skv_status;
@@ -118,11 +118,13 @@ typedef enum { SKV_HND = 0, SKV_NHD = 1, SKV_TND = 2 } skv_layout;
  * workspace: device, >= attn_fwd_lse_workspace(...) bytes, 256-byte aligned;
  *   may be NULL when that query returns 0.  After a varlen call its first
  *   bytes hold the work order: int32 order[B] (sequences, longest kv first,
- *   ties by index) then int32 offsets[B+1] (prefix sums of Hq*ceil(len_q/256)).
+ *   ties by index) then int32 offsets[B+1] (prefix sums of
+ *   Hq*ceil(len_q/rows), rows = 256 query rows per CTA for D <= 128 and 128 for
+ *   D = 256).
  * Errors: SKV_ERR_INVALID_ARG for NULL q/out, NULL k/v with keys, non-positive sizes (B, Hq,
  *   Hkv, D; Sq, Sk may be 0 in the dense case), Hq % Hkv != 0, misaligned
  *   pointers, unknown layout/dtype, or missing/extra cu_seqlens;
- *   SKV_ERR_UNSUPPORTED for D not in {64,128} or dtype fp32.
+ *   SKV_ERR_UNSUPPORTED for D not in {64,128,256} or dtype fp32.
  */
 skv_status attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
                         int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
@@ -213,9 +215,10 @@ size_t attn_fwd_lse_workspace(int B, int Hq, int Hkv, int Sk, int D, skv_dtype d
 
 /* Host restatement of the varlen work order the device builds (for tests and
  * inspection).  cu_seqlens_q/k are HOST arrays of B+1 entries; writes order[B]
- * and offsets[B+1] as documented under attn_fwd_lse with rows_per_cta = 256. */
+ * and offsets[B+1] as documented under attn_fwd_lse, for head dimension D
+ * (rows per CTA: 256 for D <= 128, 128 for D = 256). */
 skv_status attn_varlen_plan(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
-                            int Hq, int32_t* order, int32_t* offsets);
+                            int Hq, int D, int32_t* order, int32_t* offsets);
 
 /* ------------------------------------------------------------------------ */
 /* attn_splitkv_decode: split-KV decode with a stable online softmax.        */
@@ -382,8 +385,16 @@ skv_status skv_device_error(int* code);
  * devices, all threads).  Benchmarks difference it around a timed region. */
 uint64_t skv_launch_count(void);
 
-/* Library version, e.g. "0.1.0". */
+/* Library version, e.g. "0.2.0". */
 const char* skv_version(void);
+
+/* Evaluates, elementwise on the device, the exp2 that the prefill softmax
+ * computes on the FMA pipe for a share of its probabilities: y[i] = 2^x[i]
+ * from the degree-3 minimax polynomial of exp2_poly_fit.py (relative error
+ * <= 7.5e-5 for x in [-125, 126]; x < -125 gives a value below 2^-124).  Not
+ * part of the attention path (for tests of that error).  x, y: device fp32
+ * arrays of n elements. */
+skv_status skv_exp2_fma(const float* x, float* y, int64_t n, skv_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -44,7 +44,7 @@ SIGNATURES = {
                                    _c_int, _c_int, _vp, _c_size, _vp]),
     "attn_fwd_lse_int8_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "attn_fwd_lse_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
-    "attn_varlen_plan": (_c_int, [_vp, _vp, _c_int, _c_int, _vp, _vp]),
+    "attn_varlen_plan": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp]),
     "attn_splitkv_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_float, _c_int, _vp, _c_int, _vp, _c_size, _vp]),
     "attn_splitkv_decode_static": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -63,6 +63,7 @@ SIGNATURES = {
     "skv_device_error": (_c_int, [_vp]),
     "skv_version": (ctypes.c_char_p, []),
     "skv_launch_count": (ctypes.c_uint64, []),
+    "skv_exp2_fma": (_c_int, [_vp, _vp, _c_i64, _vp]),
 }
 
 _lib = None
@@ -197,20 +198,32 @@ def attn_fwd_lse_workspace(B: int, Hq: int, Hkv: int, Sk: int, D: int, dtype: st
     return int(lib().attn_fwd_lse_workspace(B, Hq, Hkv, Sk, D, DTYPES[dtype], LAYOUTS[layout], int(smooth_k)))
 
 
-def attn_varlen_plan(cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int], Hq: int) -> Tuple[list, list]:
-    """Host restatement of the device varlen work order: (order[B], offsets[B+1])."""
+def attn_varlen_plan(cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int], Hq: int,
+                     D: int = 128) -> Tuple[list, list]:
+    """Host restatement of the device varlen work order: (order[B], offsets[B+1])
+    for head dimension D (256 query rows per CTA for D <= 128, 128 for D = 256)."""
     B = len(cu_seqlens_q) - 1
     cq = (ctypes.c_int32 * (B + 1))(*[int(x) for x in cu_seqlens_q])
     ck = (ctypes.c_int32 * (B + 1))(*[int(x) for x in cu_seqlens_k])
     order = (ctypes.c_int32 * max(B, 1))()
     offsets = (ctypes.c_int32 * (B + 1))()
-    _check(lib().attn_varlen_plan(cq, ck, B, Hq, order, offsets), "attn_varlen_plan")
+    _check(lib().attn_varlen_plan(cq, ck, B, Hq, D, order, offsets), "attn_varlen_plan")
     return list(order)[:B], list(offsets)
 
 
 def launch_count() -> int:
     """Kernels launched by the library in this process so far."""
     return int(lib().skv_launch_count())
+
+
+def exp2_fma(x, stream=None):
+    """The prefill softmax's FMA-pipe exp2, elementwise on a float32 CUDA tensor (diagnostics)."""
+    torch = _torch()
+    _need_cuda(x)
+    _expect(x.dtype == torch.float32, "x must be float32")
+    y = torch.empty_like(x)
+    _check(lib().skv_exp2_fma(_ptr(x), _ptr(y), x.numel(), _stream(stream, x.device)), "skv_exp2_fma")
+    return y
 
 
 def device_error() -> int:

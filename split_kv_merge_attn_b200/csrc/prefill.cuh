@@ -7,14 +7,15 @@
 // of its 128-row tile) computes and stores row i's LSE itself.
 //
 // CTA = up to two 128-row query tiles of one (sequence, head) that share every
-// K/V tile.  Warp roles (320 threads):
+// K/V tile (one tile at D = 256).  Warp roles (320 threads):
 //   warps 0-3  softmax + epilogue for query tile 0 (thread t owns row t)
 //   warps 4-7  softmax + epilogue for query tile 1
 //   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of
 //              NS shared-memory buffers (128-byte swizzle, no multicast)
 //   warp  9    TMEM allocator and (one elected thread) tcgen05.mma issuer
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [256+D, 256+2D).  S_a holds fp32 logits; the softmax writes P_a as
+// O_1 [256+D, 256+2D) (D <= 128; at D = 256 O_0 fills [256,512) and S_1, O_1
+// are unused: the MMA order is S_0(j), PV_0(j) with the softmax between).  S_a holds fp32 logits; the softmax writes P_a as
 // packed 16-bit pairs into S_a's first 64 columns, and O_a += P_a V_j reads P_a
 // straight from TMEM (A operand in tensor memory).
 //
@@ -41,14 +42,15 @@ constexpr int kPfBN = 128;          // keys per KV tile
 constexpr int kPfThreads = 320;
 constexpr float kPfRescaleThreshold = 8.0f;
 
-// Tuning switches (compile time) of the softmax's exponent pass, which is
-// bound by the special-function unit (ex2 and the packing conversion share it):
+// Tuning switches (compile time) of the softmax's exponent pass, whose 64
+// ex2 per row half occupy the special-function unit (about 8 cycles per warp
+// instruction on B200, against 2.3 for a packed fp32 FMA):
 //   SKV_PF_POLY_PAIRS  of every 16 pairs of probabilities, this many are
 //                      computed on the FMA pipe (poly_exp2_pair) instead of ex2;
 //   SKV_PF_INT_PACK    1: round the probabilities to 16 bits with integer
 //                      operations instead of the conversion instruction.
 #ifndef SKV_PF_POLY_PAIRS
-#define SKV_PF_POLY_PAIRS 0
+#define SKV_PF_POLY_PAIRS 6   // measured best of 0, 4, 6, 8, 10 (varlen workload: 960 -> 1000 TFLOP/s)
 #endif
 #ifndef SKV_PF_INT_PACK
 #define SKV_PF_INT_PACK 0
@@ -59,7 +61,8 @@ constexpr float kPfRescaleThreshold = 8.0f;
 // of least maximum relative error on [-1/2, 1/2] (7.5e-5; the coefficients
 // are those printed by exp2_poly_fit.py in this directory, a Remez exchange);
 // 2^n is an addition to the exponent field.  Arguments below -126 are clamped
-// there (results < 2^-125).
+// there; below -125 the results are only known to be < 2^-124 (no row sum
+// notices them: the row's largest probability is >= 1).
 constexpr float kExp2C0 = 0.9999280571937561f;
 constexpr float kExp2C1 = 0.6932609677314758f;
 constexpr float kExp2C2 = 0.2426111251115799f;
@@ -130,8 +133,15 @@ __device__ __forceinline__ void s32_to_magic_64(float (&v)[64]) {
   for (int c = 0; c < 64; ++c) v[c] = __int_as_float(__float_as_int(v[c]) + 0x4B400000);
 }
 
+// Query tiles per CTA: two (the MMA ping-pongs between them) for D <= 128; one
+// for D = 256, whose O accumulator takes the 256 TMEM columns the second tile
+// would need.
+__host__ __device__ constexpr int prefill_tiles(int D) { return D == 256 ? 1 : 2; }
+
 template <int D, bool kI8 = false>
 struct PrefillCfg {
+  static constexpr int kTiles = prefill_tiles(D);
+  static constexpr int kRows = kTiles * kPfBM;       // query rows per CTA
   static constexpr int kBoxes = D / 64;              // 64-element boxes of a 16-bit row (V, and Q/K)
   static constexpr int kQKBoxes = kI8 ? D / 128 : kBoxes;  // boxes of a Q or K row
   static constexpr int kQKBoxElems = kI8 ? 128 : 64;
@@ -139,18 +149,22 @@ struct PrefillCfg {
   static constexpr int kQTileBytes = kQKBoxes * kBoxBytes;
   static constexpr int kKTileBytes = kQKBoxes * kBoxBytes;
   static constexpr int kKVTileBytes = kBoxes * kBoxBytes;   // one ring buffer (a V tile; a K tile fits)
-  static constexpr int kStages = (D == 64) ? 8 : 5;
+  // D = 256: K_j and V_j only; with one query tile, K_{j+1} loads while the
+  // softmax of step j runs and V_{j+1} while S(j+1) and that softmax run
+  static constexpr int kStages = (D == 64) ? 8 : (D == 256 ? 2 : 5);
   static constexpr int kRingBytes = kStages * kKVTileBytes;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffRing = 2 * kQTileBytes;
+  static constexpr int kOffRing = kTiles * kQTileBytes;
   static constexpr int kOffBar = kOffRing + kRingBytes;
   // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], p_half[2][2], o_full[2], drain
   static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffMu = kOffMisc + 16;             // [2][D] fp32 mean of K (smooth_k)
   static constexpr int kSmemBytes = kOffMu + 2 * D * 4 + 1024;  // + alignment pad
-  static constexpr int kSCol0 = 0, kSCol1 = 128, kOCol0 = 256, kOCol1 = 256 + D;
+  static constexpr int kSCol0 = 0, kSCol1 = 128, kOCol0 = 256, kOCol1 = 256 + D;  // O_1 only when kTiles = 2
   static constexpr uint32_t kTmemCols = 512;
+  static_assert(kOCol0 + kTiles * D <= 512, "TMEM columns");
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 struct PrefillArgs {
@@ -196,7 +210,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + Cfg::kStages;
   uint64_t* s_full = kv_empty + Cfg::kStages;
-  uint64_t* p_half = s_full + 2;     // [tile][half]: P columns of keys [64h, 64h+64) are in TMEM
+  uint64_t* p_half = s_full + 2;     // [tile][half]: P of keys [64h, 64h+64) is in TMEM (half 1 first)
   uint64_t* o_full = p_half + 4;
   uint64_t* drain = o_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
@@ -222,7 +236,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int rem = item - a.offsets[lo];
     len_q = a.cu_q[b + 1] - a.cu_q[b];
     len_k = a.cu_k[b + 1] - a.cu_k[b];
-    const int nblk = (len_q + 2 * kPfBM - 1) / (2 * kPfBM);
+    const int nblk = (len_q + Cfg::kRows - 1) / Cfg::kRows;
     if (a.causal) {
       // causal work grows with the block index: the sequence's last (longest)
       // blocks of every head start first
@@ -232,7 +246,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       h = rem / nblk;
       qblk = rem % nblk;
     }
-    q_row0 = a.cu_q[b] + qblk * 2 * kPfBM;
+    q_row0 = a.cu_q[b] + qblk * Cfg::kRows;
     k_row0 = a.cu_k[b];
     bcoord = 0;
   } else {
@@ -256,7 +270,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     len_q = a.Sq;
     len_k = a.kvb[chunk + 1] - a.kvb[chunk];
-    q_row0 = qblk * 2 * kPfBM;
+    q_row0 = qblk * Cfg::kRows;
     k_row0 = a.kvb[chunk];
     bcoord = b;
   }
@@ -265,14 +279,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int seq = b * a.nchunks + chunk;
   const int nseq = a.B * a.nchunks;
   const int hkv = h / G;
-  const int rows_here = min(2 * kPfBM, len_q - qblk * 2 * kPfBM);
+  const int rows_here = min(Cfg::kRows, len_q - qblk * Cfg::kRows);
   const int nt = rows_here > kPfBM ? 2 : 1;
   // causal: rows are the last len_q positions of the key range (bottom-right
   // alignment); the block stops at the KV tile holding its last row's last
   // key, and both query tiles run over the same tiles (the first tile's rows
   // simply see more masked keys)
   const int causal_off = len_k - len_q;
-  const int kv_end = a.causal ? min(max(qblk * 2 * kPfBM + rows_here + causal_off, 0), len_k) : len_k;
+  const int kv_end = a.causal ? min(max(qblk * Cfg::kRows + rows_here + causal_off, 0), len_k) : len_k;
   const int nkv = (kv_end + kPfBN - 1) / kPfBN;
 
   // output addressing for query row qi (index inside the sequence); the rows
@@ -293,7 +307,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   if (nkv == 0) {
     // no keys: O = 0, LSE = -inf for every valid row of this block
     for (int r = tid; r < rows_here; r += kPfThreads) {
-      const int qi = qblk * 2 * kPfBM + r;
+      const int qi = qblk * Cfg::kRows + r;
       uint4* dst = reinterpret_cast<uint4*>(out_row(qi));
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
@@ -409,14 +423,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         __syncwarp();
       };
+      // PV over the 64 keys of half hf: key block kk (16 keys) reads P from
+      // columns kk * 8 (half 0) or 64 + (kk - 4) * 8 (half 1), where the
+      // softmax writes them; half 1 is issued first, so its first MMA is the
+      // one that overwrites O when `acc` is false
       auto issue_pv_half = [&](uint32_t sc, uint32_t oc, int u, bool acc, int hf) {
         const uint64_t dv = dv_base + static_cast<uint64_t>(((u % Cfg::kStages) * Cfg::kKVTileBytes) >> 4);
         if (elect_one()) {
 #pragma unroll
           for (int k4 = 0; k4 < kPfBN / 32; ++k4) {
             const int kk = hf * (kPfBN / 32) + k4;
-            tc5::mma_ts(oc, sc + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
-                        (acc || kk > 0) ? 1u : 0u);
+            tc5::mma_ts(oc, sc + kk * 8 + hf * 32, dv + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
+                        (acc || hf == 0 || k4 > 0) ? 1u : 0u);
           }
         }
         __syncwarp();
@@ -433,14 +451,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       };
       auto wait_kv = [&](int u) -> bool { return wait_bar(&kv_full[u % Cfg::kStages], (u / Cfg::kStages) & 1); };
       auto wait_p = [&](int t, int hf, int j) -> bool { return wait_bar(&p_half[2 * t + hf], j & 1); };
-      // PV of tile t for KV tile j, started on the first 64 keys of P while the
-      // softmax still exponentiates the second 64
+      // PV of tile t for KV tile j, started on keys [64, 128) of P while the
+      // softmax still exponentiates keys [0, 64)
       auto issue_pv = [&](int t, int u, bool acc, int j) -> bool {
         const uint32_t sc = t ? s1c : s0c, oc = t ? o1c : o0c;
-        if (!wait_p(t, 0, j)) return false;
-        issue_pv_half(sc, oc, u, acc, 0);
         if (!wait_p(t, 1, j)) return false;
         issue_pv_half(sc, oc, u, acc, 1);
+        if (!wait_p(t, 0, j)) return false;
+        issue_pv_half(sc, oc, u, acc, 0);
         return true;
       };
       auto release = [&](int u) { commit(&kv_empty[u % Cfg::kStages]); };
@@ -488,7 +506,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint32_t lane_base = static_cast<uint32_t>(lg * 32) << 16;
       const uint32_t s_addr = tmem + lane_base + (t == 0 ? Cfg::kSCol0 : Cfg::kSCol1);
       const uint32_t o_addr = tmem + lane_base + (t == 0 ? Cfg::kOCol0 : Cfg::kOCol1);
-      const int qi = qblk * 2 * kPfBM + t * kPfBM + row;  // row index inside the sequence
+      const int qi = qblk * Cfg::kRows + t * kPfBM + row;  // row index inside the sequence
       const bool row_valid = qi < len_q;
       const int row_keys = a.causal ? min(max(qi + causal_off + 1, 0), len_k) : len_k;  // keys this row sees
       bool ok = true;
@@ -500,12 +518,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (a.kpartial != nullptr) {
           // mean over this call's KV range from the per-256-key column sums
           float* mu_s = reinterpret_cast<float*>(smem + Cfg::kOffMu) + t * D;
-          if (row < D) {
+          for (int d = row; d < D; d += kPfBM) {
             const int nch = (len_k + 255) / 256;
             float sum = 0.f;
             for (int c = 0; c < nch; ++c)
-              sum += __ldg(a.kpartial + ((static_cast<int64_t>(c) * nseq + seq) * a.Hkv + hkv) * D + row);
-            mu_s[row] = sum / static_cast<float>(len_k);
+              sum += __ldg(a.kpartial + ((static_cast<int64_t>(c) * nseq + seq) * a.Hkv + hkv) * D + d);
+            mu_s[d] = sum / static_cast<float>(len_k);
           }
           named_barrier_sync(1 + t, kPfBM);
           mu = mu_s;
@@ -559,14 +577,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           sl2 = a.scale_log2 * qsc * ks_next;
           if (j + 1 < nkv) ks_next = __ldg(ksc + j + 1);
         }
-        // pass 1 over S (two halves of 64 columns read from TMEM): the row max
+        // pass 1 over S (two halves of 64 columns read from TMEM): the row max;
+        // the second half's logits stay in sh for the exponent pass
         const int n_valid = row_keys - j * kPfBN;
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+        float sh[64];
 #pragma unroll 1
         for (int hf = 0; hf < 2; ++hf) {
-          float sh[64];
           tc5::ld32(s_addr + hf * 64, *reinterpret_cast<float(*)[32]>(&sh[0]));
           tc5::ld32(s_addr + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
           tc5::wait_ld();
@@ -610,38 +629,45 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
           tc5::wait_st();
         }
-        // p = 2^(s * scale*log2(e) - max): P of keys [64h, 64h+64) is packed into
-        // columns [32h, 32h+32) (logits this thread has already read) and
-        // published on its own barrier, so PV can start on the first half
-        // a row that has seen no key yet (causal rows before the first key)
-        // keeps m = -inf: exponentiate its masked logits against 0 instead
+        // p = 2^(s * scale*log2(e) - max), packed as 16-bit pairs into TMEM and
+        // published per 64-key half on its own barrier, so PV starts on one half
+        // while the other is exponentiated.  Keys [64, 128) go first, from the
+        // registers of the max pass; their P lands in columns [64, 96) (logits
+        // already read).  Keys [0, 64) are then reloaded (the load is issued
+        // before the first half's store is waited for) and their P lands in
+        // columns [0, 32).
+        // A row that has seen no key yet (causal rows before the first key)
+        // keeps m = -inf: exponentiate its masked logits against 0 instead.
         float neg_bias = -((m_run == -INFINITY ? 0.f : m_run) + bias_shift);
         if constexpr (kI8) neg_bias = fmaf(-kMagic, sl2, neg_bias);  // the logits carry +kMagic
         const uint64_t sc2 = f2_pack(sl2, sl2);
         const uint64_t nb2 = f2_pack(neg_bias, neg_bias);
         uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
         const bool full_tile = n_valid >= kPfBN;
-#pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-          float sh[64];
-          tc5::ld32(s_addr + hf * 64, *reinterpret_cast<float(*)[32]>(&sh[0]));
-          tc5::ld32(s_addr + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
-          tc5::wait_ld();
-          if constexpr (kI8) s32_to_magic_64(sh);
-          if (!full_tile) {
+        uint32_t pk[32];
+        if (full_tile) exp_pack_64<true, T>(sh, sc2, nb2, pk, ps2);
+        else exp_pack_64<false, T>(sh, sc2, nb2, pk, ps2);
+        tc5::st16(s_addr + 64, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+        tc5::st16(s_addr + 80, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+        tc5::ld32(s_addr, *reinterpret_cast<float(*)[32]>(&sh[0]));
+        tc5::ld32(s_addr + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
+        tc5::wait_st();
+        tc5::fence_before();
+        mbar_arrive(&p_half[2 * t + 1]);
+        tc5::wait_ld();
+        if constexpr (kI8) s32_to_magic_64(sh);
+        if (!full_tile) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (hf * 64 + c >= n_valid) sh[c] = -INFINITY;
-          }
-          uint32_t pk[32];
-          if (full_tile) exp_pack_64<true, T>(sh, sc2, nb2, pk, ps2);
-          else exp_pack_64<false, T>(sh, sc2, nb2, pk, ps2);
-          tc5::st16(s_addr + hf * 32, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-          tc5::st16(s_addr + hf * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
-          tc5::wait_st();
-          tc5::fence_before();
-          mbar_arrive(&p_half[2 * t + hf]);
+          for (int c = 0; c < 64; ++c)
+            if (c >= n_valid) sh[c] = -INFINITY;
         }
+        if (full_tile) exp_pack_64<true, T>(sh, sc2, nb2, pk, ps2);
+        else exp_pack_64<false, T>(sh, sc2, nb2, pk, ps2);
+        tc5::st16(s_addr, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+        tc5::st16(s_addr + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+        tc5::wait_st();
+        tc5::fence_before();
+        mbar_arrive(&p_half[2 * t + 0]);
         const float2 psa = f2_unpack(ps2[0]), psb = f2_unpack(ps2[1]);
         l_run += (psa.x + psa.y) + (psb.x + psb.y);
       }
@@ -682,7 +708,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // error word says so
       named_barrier_sync(1 + t, kPfBM);
       if (ok) {
-        const int row0 = qblk * 2 * kPfBM + t * kPfBM;
+        const int row0 = qblk * Cfg::kRows + t * kPfBM;
 #pragma unroll 4
         for (int i = 0; i < kChunks; ++i) {
           const int idx = i * kPfBM + row;
@@ -706,9 +732,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
 // Device-side varlen planner (one block): orders sequences by kv length,
 // longest first (ties by index), and writes prefix sums of their work items
-// (Hq * ceil(len_q / 256)).  order[B], offsets[B+1].
+// (Hq * ceil(len_q / rows_per_cta)).  order[B], offsets[B+1].
 __global__ void __launch_bounds__(1024) varlen_plan_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k,
-                                                            int B, int Hq, int* __restrict__ order,
+                                                            int B, int Hq, int rows_per_cta, int* __restrict__ order,
                                                             int* __restrict__ offsets) {
   for (int bb = threadIdx.x; bb < B; bb += blockDim.x) {
     const int lk = cu_k[bb + 1] - cu_k[bb];
@@ -729,7 +755,7 @@ __global__ void __launch_bounds__(1024) varlen_plan_kernel(const int* __restrict
   for (int i = beg; i < end; ++i) {
     const int bb = order[i];
     const int lq = cu_q[bb + 1] - cu_q[bb];
-    local += Hq * ((lq + 2 * kPfBM - 1) / (2 * kPfBM));
+    local += Hq * ((lq + rows_per_cta - 1) / rows_per_cta);
   }
   part[threadIdx.x] = local;
   __syncthreads();
@@ -748,7 +774,7 @@ __global__ void __launch_bounds__(1024) varlen_plan_kernel(const int* __restrict
     offsets[i] = run;
     const int bb = order[i];
     const int lq = cu_q[bb + 1] - cu_q[bb];
-    run += Hq * ((lq + 2 * kPfBM - 1) / (2 * kPfBM));
+    run += Hq * ((lq + rows_per_cta - 1) / rows_per_cta);
   }
 }
 

@@ -101,7 +101,12 @@ const char* skv_status_string(skv_status s) {
 
 int skv_last_cuda_error(void) { return g_last_cuda_error; }
 
-const char* skv_version(void) { return "0.1.0"; }
+const char* skv_version(void) { return "0.2.0"; }
+
+skv_status skv_exp2_fma(const float* x, float* y, int64_t n, skv_stream_t stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return SKV_ERR_INVALID_ARG;
+  return cuda_status(skv::launch_exp2_fma(x, y, n, stream));
+}
 
 uint64_t skv_launch_count(void) { return skv::launch_count(); }
 
@@ -154,10 +159,11 @@ size_t attn_splitkv_workspace(int B, int Hq, int Lq, int D, int num_splits) {
   return decode_workspace(B, Hq, Lq, D, num_splits);
 }
 
-skv_status attn_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int32_t* order,
+skv_status attn_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int D, int32_t* order,
                             int32_t* offsets) {
-  if (cu_q == nullptr || cu_k == nullptr || order == nullptr || offsets == nullptr || B < 1 || Hq < 1)
+  if (cu_q == nullptr || cu_k == nullptr || order == nullptr || offsets == nullptr || B < 1 || Hq < 1 || D < 1)
     return SKV_ERR_INVALID_ARG;
+  const int rows = skv::prefill_rows_per_cta(D);
   for (int b = 0; b < B; ++b)
     if (cu_q[b + 1] < cu_q[b] || cu_k[b + 1] < cu_k[b]) return SKV_ERR_INVALID_ARG;
   std::vector<int> idx(B);
@@ -170,7 +176,7 @@ skv_status attn_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int
     order[i] = idx[i];
     offsets[i] = static_cast<int32_t>(run);
     const int64_t lq = cu_q[idx[i] + 1] - cu_q[idx[i]];
-    run += static_cast<int64_t>(Hq) * skv::ceil_div64(lq, skv::kPrefillRowsPerCta);
+    run += static_cast<int64_t>(Hq) * skv::ceil_div64(lq, rows);
   }
   offsets[B] = static_cast<int32_t>(run);
   return SKV_OK;
@@ -213,7 +219,7 @@ skv_status fwd_lse_impl(const void* q, const void* k, const void* v, void* out, 
     if (cu_seqlens_q != nullptr || cu_seqlens_k != nullptr) return SKV_ERR_INVALID_ARG;
   }
   if (!is_half_type(dtype)) return SKV_ERR_UNSUPPORTED;
-  if (D != 64 && D != 128) return SKV_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128 && D != 256) return SKV_ERR_UNSUPPORTED;
   // TMA extents and int32 coordinates
   const int64_t rows_q = varlen ? Sq : static_cast<int64_t>(Sq);
   if (rows_q > (int64_t(1) << 31) - 512 || Sk > (1 << 30)) return SKV_ERR_UNSUPPORTED;
@@ -228,8 +234,7 @@ skv_status fwd_lse_impl(const void* q, const void* k, const void* v, void* out, 
       max_chunk = std::max(max_chunk, kv_bounds[c + 1] - kv_bounds[c]);
     }
     // every chunk's partial is one output's worth of rows further
-    if (static_cast<int64_t>(nchunks) * B * Hq * ((Sq + skv::kPrefillRowsPerCta - 1) / skv::kPrefillRowsPerCta) >
-        0x7fffffff)
+    if (static_cast<int64_t>(nchunks) * B * Hq * skv::ceil_div64(Sq, skv::prefill_rows_per_cta(D)) > 0x7fffffff)
       return SKV_ERR_UNSUPPORTED;
   }
   const FwdWorkspace ws = fwd_workspace(B, Hkv, Sk, D, layout, smooth_k, nchunks);
@@ -263,7 +268,8 @@ skv_status fwd_lse_impl(const void* q, const void* k, const void* v, void* out, 
     p.cu_k = cu_seqlens_k;
     p.order = reinterpret_cast<const int32_t*>(wsb + ws.order);
     p.offsets = reinterpret_cast<const int32_t*>(wsb + ws.offsets);
-    int e = skv::launch_varlen_plan(cu_seqlens_q, cu_seqlens_k, B, Hq, reinterpret_cast<int32_t*>(wsb + ws.order),
+    int e = skv::launch_varlen_plan(cu_seqlens_q, cu_seqlens_k, B, Hq, skv::prefill_rows_per_cta(D),
+                                    reinterpret_cast<int32_t*>(wsb + ws.order),
                                     reinterpret_cast<int32_t*>(wsb + ws.offsets), stream);
     if (e) return cuda_status(e);
   }

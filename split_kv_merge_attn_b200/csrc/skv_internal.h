@@ -32,7 +32,9 @@ constexpr int kCtasPerSmD256Num = 2, kCtasPerSmD256Den = 3;
 constexpr int kDecodeRowsPerCta = 16;
 // Largest number of KV chunks of one multi-chunk prefill call.
 constexpr int kMaxKvChunks = 64;
-constexpr int kPrefillRowsPerCta = 256;
+constexpr int kPrefillRowsPerCta = 256;      // two 128-row query tiles (D <= 128)
+constexpr int kPrefillRowsPerCtaD256 = 128;  // one tile (D = 256)
+inline int prefill_rows_per_cta(int D) { return D == 256 ? kPrefillRowsPerCtaD256 : kPrefillRowsPerCta; }
 
 inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -98,7 +100,7 @@ struct Int8PrefillLaunch {
 };
 int launch_prefill_int8(const Int8PrefillLaunch& p, skv_stream_t stream);
 
-int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int32_t* order,
+int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int rows_per_cta, int32_t* order,
                        int32_t* offsets, skv_stream_t stream);
 
 // smooth_k prepass: fp32 per-256-key column sums of K for each (batch or
@@ -111,6 +113,9 @@ int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partia
                     int kv_ranges = 1, const int32_t* kv_bounds = nullptr);
 
 int read_and_clear_device_error(int* code);
+
+// Elementwise evaluation of the prefill's FMA-pipe exp2 (diagnostics).
+int launch_exp2_fma(const float* x, float* y, int64_t n, skv_stream_t stream);
 
 // Maps a cudaError_t value to a status: SKV_OK for 0, else SKV_ERR_CUDA with
 // the error recorded for skv_last_cuda_error on the calling thread.

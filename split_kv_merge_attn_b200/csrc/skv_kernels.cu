@@ -16,7 +16,14 @@
 #include "decode.cuh"
 #include "quant.cuh"
 #include "prefill.cuh"
+#include "prefill_db.cuh"
 #include "smooth.cuh"
+
+// Tuning switch: 1 = 16-bit prefill at D <= 128 runs prefill_db_kernel (two S
+// buffers per query tile, 64-key steps); 0 = prefill_kernel (128-key steps).
+#ifndef SKV_PF_DB
+#define SKV_PF_DB 0
+#endif
 
 namespace skv {
 
@@ -270,19 +277,20 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
 
 namespace {
 // 4-D map over q/k/v of one layout: HND dims (D, S, H, B); NHD / TND dims
-// (D, H, S, B); box = 64 columns x 128 rows of one head.
-int make_qkv_map(CUtensorMap* m, const void* base, skv_dtype dt, skv_layout layout, int B, int H, int S, int D) {
+// (D, H, S, B); box = 64 columns x `rows` rows of one head.
+int make_qkv_map(CUtensorMap* m, const void* base, skv_dtype dt, skv_layout layout, int B, int H, int S, int D,
+                 uint32_t rows = 128) {
   const uint64_t e = 2;
   uint64_t dims[4], strides[3];
   uint32_t box[4];
   if (layout == SKV_HND) {
     dims[0] = D; dims[1] = S; dims[2] = H; dims[3] = B;
     strides[0] = D * e; strides[1] = static_cast<uint64_t>(S) * D * e; strides[2] = static_cast<uint64_t>(H) * S * D * e;
-    box[0] = 64; box[1] = 128; box[2] = 1; box[3] = 1;
+    box[0] = 64; box[1] = rows; box[2] = 1; box[3] = 1;
   } else {
     dims[0] = D; dims[1] = H; dims[2] = S; dims[3] = B;
     strides[0] = D * e; strides[1] = static_cast<uint64_t>(H) * D * e; strides[2] = static_cast<uint64_t>(S) * H * D * e;
-    box[0] = 64; box[1] = 1; box[2] = 128; box[3] = 1;
+    box[0] = 64; box[1] = 1; box[2] = rows; box[3] = 1;
   }
   return make_tmap(m, dt, 4, base, dims, strides, box);
 }
@@ -306,20 +314,32 @@ int launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   kern<<<grid, kPfThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, a);
   return counted(cudaGetLastError(), 1);
 }
+
+template <int D, typename T>
+int launch_prefill_db_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillArgs& a,
+                        unsigned grid, cudaStream_t st) {
+  using Cfg = PfDbCfg<D>;
+  auto kern = prefill_db_kernel<D, T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kPfThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, a);
+  return counted(cudaGetLastError(), 1);
+}
 }  // namespace
 
 int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   const bool varlen = p.layout == SKV_TND;
   const int Bm = varlen ? 1 : p.B;       // batch extent of the maps
+  const bool db = SKV_PF_DB && p.D <= 128;  // 64-key K/V tiles
   CUtensorMap tq, tk, tv;
   int e = make_qkv_map(&tq, p.q, p.dt, p.layout, Bm, p.Hq, p.Sq > 0 ? p.Sq : 1, p.D);
   if (e) return e;
   std::memset(&tk, 0, sizeof(tk));
   std::memset(&tv, 0, sizeof(tv));
   if (p.Sk > 0) {  // with no keys every CTA writes O = 0, LSE = -inf without loads
-    e = make_qkv_map(&tk, p.k, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D);
+    e = make_qkv_map(&tk, p.k, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D, db ? kDbBN : 128);
     if (e) return e;
-    e = make_qkv_map(&tv, p.v, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D);
+    e = make_qkv_map(&tv, p.v, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D, db ? kDbBN : 128);
     if (e) return e;
   }
   PrefillArgs a;
@@ -354,20 +374,32 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   if (varlen) {
     // upper bound on sum_b ceil(len_q(b) / 256); surplus CTAs exit at once
     a.nqb = 0;
-    grid = static_cast<int64_t>(p.Hq) * (ceil_div64(p.Sq, kPrefillRowsPerCta) + p.B);
+    grid = static_cast<int64_t>(p.Hq) * (ceil_div64(p.Sq, prefill_rows_per_cta(p.D)) + p.B);
   } else {
-    a.nqb = static_cast<int>(ceil_div64(p.Sq, kPrefillRowsPerCta));
+    a.nqb = static_cast<int>(ceil_div64(p.Sq, prefill_rows_per_cta(p.D)));
     grid = static_cast<int64_t>(nch) * p.B * p.Hq * a.nqb;
   }
   if (grid <= 0) return 0;
   if (grid > 0x7fffffff) return cudaErrorInvalidValue;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (db) {
+    if (p.dt == SKV_BF16) {
+      if (p.D == 64) return launch_prefill_db_t<64, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+      if (p.D == 128) return launch_prefill_db_t<128, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+    } else {
+      if (p.D == 64) return launch_prefill_db_t<64, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+      if (p.D == 128) return launch_prefill_db_t<128, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+    }
+    return cudaErrorInvalidValue;
+  }
   if (p.dt == SKV_BF16) {
     if (p.D == 64) return launch_prefill_t<64, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
     if (p.D == 128) return launch_prefill_t<128, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+    if (p.D == 256) return launch_prefill_t<256, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
   } else {
     if (p.D == 64) return launch_prefill_t<64, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
     if (p.D == 128) return launch_prefill_t<128, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+    if (p.D == 256) return launch_prefill_t<256, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
   }
   return cudaErrorInvalidValue;
 }
@@ -462,12 +494,41 @@ int launch_prefill_int8(const Int8PrefillLaunch& p, skv_stream_t stream) {
   return launch_prefill_t<128, __half, true>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
 }
 
-int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int32_t* order, int32_t* offsets,
-                       skv_stream_t stream) {
+int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int rows_per_cta, int32_t* order,
+                       int32_t* offsets, skv_stream_t stream) {
   // one block; no more threads than sequences (rounded to a warp): the final
   // scan walks one partial sum per thread
   const int threads = B >= 1024 ? 1024 : ((B + 31) / 32) * 32;
-  varlen_plan_kernel<<<1, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(cu_q, cu_k, B, Hq, order, offsets);
+  varlen_plan_kernel<<<1, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(cu_q, cu_k, B, Hq, rows_per_cta, order,
+                                                                               offsets);
+  return counted(cudaGetLastError(), 1);
+}
+
+// ------------------------------------------------------------ diagnostics
+
+namespace {
+// The prefill's FMA-pipe exp2, elementwise (for tests of its error).
+__global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (2 * i + 1 < n) {
+    float p0, p1;
+    poly_exp2_pair(f2_pack(x[2 * i], x[2 * i + 1]), p0, p1);
+    y[2 * i] = p0;
+    y[2 * i + 1] = p1;
+  } else if (2 * i < n) {
+    float p0, p1;
+    poly_exp2_pair(f2_pack(x[2 * i], 0.f), p0, p1);
+    y[2 * i] = p0;
+  }
+}
+}  // namespace
+
+int launch_exp2_fma(const float* x, float* y, int64_t n, skv_stream_t stream) {
+  const int64_t pairs = (n + 1) / 2;
+  if (pairs == 0) return 0;
+  const int64_t blocks = (pairs + 255) / 256;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  exp2_fma_kernel<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
   return counted(cudaGetLastError(), 1);
 }
 

@@ -74,7 +74,6 @@ def test_attn_fwd_lse_rejects_invalid_arguments():
     assert fwd(cq=P16, ck=P16) == INVALID              # cu_seqlens with a dense layout
     assert fwd(layout=2) == INVALID                    # varlen without cu_seqlens
     assert fwd(layout=2, cq=P16, ck=P16, mq=65, Sq=64) == INVALID   # max_seqlen_q > total_q
-    assert fwd(D=256) == UNSUPPORTED
     assert fwd(D=96) == UNSUPPORTED
     assert fwd(dt=2) == UNSUPPORTED
     need = skv.attn_fwd_lse_workspace(1, 4, 4, 64, 128, "bf16", "HND", 1)
@@ -209,6 +208,9 @@ def test_varlen_plan_matches_oracle_bit_exact():
         H = int(rng.integers(1, 33))
         order, offsets, _ = O.varlen_schedule(cq, ck, H)
         assert skv.attn_varlen_plan(cq, ck, H) == (order, offsets)
+        # D = 256 runs one 128-row query tile per CTA
+        order, offsets, _ = O.varlen_schedule(cq, ck, H, rows_per_cta=128)
+        assert skv.attn_varlen_plan(cq, ck, H, D=256) == (order, offsets)
 
 
 def test_fwd_workspace_sizes():
