@@ -591,7 +591,7 @@ def run_e2e(args, dev, host, skv, torch, step_flops, world, dist):
 def kernel_source_hash() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("prefill.cuh", "prefill_db.cuh", "tcgen05.cuh", "skv_device.cuh", "skv_kernels.cu"):
+    for f in ("prefill.cuh", "tcgen05.cuh", "skv_device.cuh", "skv_kernels.cu"):
         h.update(open(os.path.join(ROOT, "split_kv_merge_attn_b200", "csrc", f), "rb").read())
     return h.hexdigest()
 

@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libsplitkv.so")
 
 SOURCES = ["skv_kernels.cu", "skv_abi.cpp", "skv_noalloc.cu"]
-HEADERS = ["skv_device.cuh", "skv_internal.h", "merge_state.cuh", "decode.cuh", "prefill.cuh", "prefill_db.cuh",
+HEADERS = ["skv_device.cuh", "skv_internal.h", "merge_state.cuh", "decode.cuh", "prefill.cuh",
            "smooth.cuh", "tcgen05.cuh", "quant.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

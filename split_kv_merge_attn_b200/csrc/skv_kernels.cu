@@ -16,14 +16,7 @@
 #include "decode.cuh"
 #include "quant.cuh"
 #include "prefill.cuh"
-#include "prefill_db.cuh"
 #include "smooth.cuh"
-
-// Tuning switch: 1 = 16-bit prefill at D <= 128 runs prefill_db_kernel (two S
-// buffers per query tile, 64-key steps); 0 = prefill_kernel (128-key steps).
-#ifndef SKV_PF_DB
-#define SKV_PF_DB 0
-#endif
 
 namespace skv {
 
@@ -315,31 +308,20 @@ int launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   return counted(cudaGetLastError(), 1);
 }
 
-template <int D, typename T>
-int launch_prefill_db_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillArgs& a,
-                        unsigned grid, cudaStream_t st) {
-  using Cfg = PfDbCfg<D>;
-  auto kern = prefill_db_kernel<D, T>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  kern<<<grid, kPfThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, a);
-  return counted(cudaGetLastError(), 1);
-}
 }  // namespace
 
 int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   const bool varlen = p.layout == SKV_TND;
   const int Bm = varlen ? 1 : p.B;       // batch extent of the maps
-  const bool db = SKV_PF_DB && p.D <= 128;  // 64-key K/V tiles
   CUtensorMap tq, tk, tv;
   int e = make_qkv_map(&tq, p.q, p.dt, p.layout, Bm, p.Hq, p.Sq > 0 ? p.Sq : 1, p.D);
   if (e) return e;
   std::memset(&tk, 0, sizeof(tk));
   std::memset(&tv, 0, sizeof(tv));
   if (p.Sk > 0) {  // with no keys every CTA writes O = 0, LSE = -inf without loads
-    e = make_qkv_map(&tk, p.k, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D, db ? kDbBN : 128);
+    e = make_qkv_map(&tk, p.k, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D);
     if (e) return e;
-    e = make_qkv_map(&tv, p.v, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D, db ? kDbBN : 128);
+    e = make_qkv_map(&tv, p.v, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D);
     if (e) return e;
   }
   PrefillArgs a;
@@ -382,16 +364,6 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   if (grid <= 0) return 0;
   if (grid > 0x7fffffff) return cudaErrorInvalidValue;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (db) {
-    if (p.dt == SKV_BF16) {
-      if (p.D == 64) return launch_prefill_db_t<64, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
-      if (p.D == 128) return launch_prefill_db_t<128, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
-    } else {
-      if (p.D == 64) return launch_prefill_db_t<64, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
-      if (p.D == 128) return launch_prefill_db_t<128, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
-    }
-    return cudaErrorInvalidValue;
-  }
   if (p.dt == SKV_BF16) {
     if (p.D == 64) return launch_prefill_t<64, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
     if (p.D == 128) return launch_prefill_t<128, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
