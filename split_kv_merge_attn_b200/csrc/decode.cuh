@@ -34,6 +34,7 @@ constexpr int kDecodeRows = 16;
 constexpr int kDecodeConsumerWarps = 4;
 constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;
 constexpr int kSplitMaxDevice = 256;   // largest num_splits (the host planner's cap)
+constexpr int kDecodeCombineHeader = 1024;  // per-warp running max and sum, before the fragments
 constexpr int kMergeStageOffset = kSplitMaxDevice * kDecodeRows * 4 + 128;  // after weights + 1/sum
 
 // Tuning switches (compile time): K/V ring depth of the decode for D = 128 and
@@ -53,7 +54,7 @@ struct DecodeCfg {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kQStride = D + 8;                      // elements; 16-byte pad per row
   static constexpr int kRingBytes = kStages * kStageBytes;
-  static constexpr int kCombineBytes = kDecodeConsumerWarps * kDecodeRows * (D + 2) * 4;
+  static constexpr int kCombineBytes = kDecodeCombineHeader + kDecodeConsumerWarps * kDecodeRows * D * 4;
   static_assert(kRingBytes >= kCombineBytes, "combine area reuses the ring");
   static constexpr int kQBytes = kDecodeRows * kQStride * 2;
   static constexpr int kSmemBytes = kRingBytes + kQBytes + 2 * kStages * 8 + 16 + 1024;  // +align pad
@@ -180,71 +181,6 @@ __device__ __forceinline__ void decode_merge_group(const DecodeArgs& a, uint8_t*
       u.y = pack2<T>(acc[j].z * inv, acc[j].w * inv);
       *reinterpret_cast<uint2*>(out + static_cast<int64_t>(v) * 4) = u;
     }
-  }
-}
-
-// Final (one split) or partial (split > 1) result of rows r of this CTA's
-// group from the four consumer warps' states; 8 threads per row, each a D/8
-// slice.
-template <int D, typename T>
-__device__ __forceinline__ void decode_write_rows(const DecodeArgs& a, const float* cm, const float* cl,
-                                                  const float* co, int b, int hkv, int G, int rglob, int r, int sl,
-                                                  int split) {
-  float M = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < kDecodeConsumerWarps; ++w) M = fmaxf(M, cm[w * 16 + r]);
-  float e[kDecodeConsumerWarps];
-  float L = 0.f;
-#pragma unroll
-  for (int w = 0; w < kDecodeConsumerWarps; ++w) {
-    const float mw = cm[w * 16 + r];
-    e[w] = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
-    L += e[w] * cl[w * 16 + r];
-  }
-  const float inv = (L > 0.f) ? 1.0f / L : 0.f;
-  const float lse_val = (L > 0.f) ? M + __log2f(L) : -INFINITY;
-  const int h = hkv * G + rglob / a.Lq;
-  const int i = rglob % a.Lq;
-  const int64_t orow = (static_cast<int64_t>(b) * a.Hq + h) * a.Lq + i;
-  const int64_t rows_all = static_cast<int64_t>(a.B) * a.Hq * a.Lq;
-  constexpr int per = D / 8;
-  if (a.num_splits == 1) {
-    T* dst = static_cast<T*>(a.out) + orow * D + sl * per;
-#pragma unroll
-    for (int c = 0; c < per; c += 8) {
-      float v[8];
-#pragma unroll
-      for (int q2 = 0; q2 < 8; ++q2) {
-        const int d = sl * per + c + q2;
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecodeConsumerWarps; ++w) acc = fmaf(e[w], co[(w * 16 + r) * D + d], acc);
-        v[q2] = acc * inv;
-      }
-      uint4 u;
-      u.x = pack2<T>(v[0], v[1]);
-      u.y = pack2<T>(v[2], v[3]);
-      u.z = pack2<T>(v[4], v[5]);
-      u.w = pack2<T>(v[6], v[7]);
-      *reinterpret_cast<uint4*>(dst + c) = u;
-    }
-    if (sl == 0 && a.lse != nullptr) a.lse[orow] = lse_val;
-  } else {
-    float* dst = a.part_o + (static_cast<int64_t>(split) * rows_all + orow) * D + sl * per;
-#pragma unroll
-    for (int c = 0; c < per; c += 4) {
-      float v[4];
-#pragma unroll
-      for (int q2 = 0; q2 < 4; ++q2) {
-        const int d = sl * per + c + q2;
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecodeConsumerWarps; ++w) acc = fmaf(e[w], co[(w * 16 + r) * D + d], acc);
-        v[q2] = acc * inv;
-      }
-      *reinterpret_cast<float4*>(dst + c) = make_float4(v[0], v[1], v[2], v[3]);
-    }
-    if (sl == 0) a.part_lse[static_cast<int64_t>(split) * rows_all + orow] = lse_val;
   }
 }
 
@@ -492,9 +428,13 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
   lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], 2);
   lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], 1);
   lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], 2);
+  // Each warp stores its accumulator fragments in fragment order: per 8-column
+  // block j one float4 per lane (rows g and g + 8, columns 2tq and 2tq + 1),
+  // so every store and every load below is a contiguous 512-byte run per warp
+  // instruction (no shared-memory bank conflicts).
   float* cm = reinterpret_cast<float*>(ring);                    // [4][16] running max
   float* cl = cm + kDecodeConsumerWarps * kDecodeRows;            // [4][16] sums
-  float* co = cl + kDecodeConsumerWarps * kDecodeRows;            // [4][16][D] accumulators
+  float4* co4 = reinterpret_cast<float4*>(ring + kDecodeCombineHeader);  // [4][D/8][32]
   if (tq == 0) {
     cm[warp * 16 + g] = m[0];
     cm[warp * 16 + g + 8] = m[1];
@@ -502,18 +442,69 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
     cl[warp * 16 + g + 8] = lsum[1];
   }
 #pragma unroll
-  for (int j = 0; j < D / 8; ++j) {
-    const int d = j * 8 + 2 * tq;
-    *reinterpret_cast<float2*>(co + (warp * 16 + g) * D + d) = make_float2(o[j][0], o[j][1]);
-    *reinterpret_cast<float2*>(co + (warp * 16 + g + 8) * D + d) = make_float2(o[j][2], o[j][3]);
-  }
+  for (int j = 0; j < D / 8; ++j) co4[(warp * (D / 8) + j) * 32 + lane] = make_float4(o[j][0], o[j][1], o[j][2], o[j][3]);
   named_barrier_sync(1, kDecodeConsumerWarps * 32);
 
-  // 128 threads: 8 per row, each a D/8 slice
-  const int r = tid >> 3;
-  const int sl = tid & 7;
-  const int rglob = rg * kDecodeRows + r;
-  if (!aborted && rglob < rows_total) decode_write_rows<D, T>(a, cm, cl, co, b, hkv, G, rglob, r, sl, split);
+  // Thread t combines fragment slots t, t + 128, ...: blocks j = warp + 4k of
+  // lane `lane`, i.e. always rows g and g + 8, whose weights it computes
+  // itself.  Per row: M = max_w m_w, L = sum_w 2^(m_w - M) l_w, weight of warp
+  // w 2^(m_w - M) / L (0 for a warp that saw no key), LSE = M + log2 L.
+  const int rows_here = min(kDecodeRows, rows_total - rg * kDecodeRows);
+  const int64_t rows_all = static_cast<int64_t>(a.B) * a.Hq * a.Lq;
+  const int64_t orow0 = (static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(hkv) * G) * a.Lq +
+                        static_cast<int64_t>(rg) * kDecodeRows;
+  if (!aborted && g < rows_here) {
+    float wt[2][kDecodeConsumerWarps];
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int r = g + 8 * hr;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kDecodeConsumerWarps; ++w) M = fmaxf(M, cm[w * 16 + r]);
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecodeConsumerWarps; ++w) {
+        const float mw = cm[w * 16 + r];
+        wt[hr][w] = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
+        L += wt[hr][w] * cl[w * 16 + r];
+      }
+      const float inv = (L > 0.f) ? 1.0f / L : 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecodeConsumerWarps; ++w) wt[hr][w] *= inv;
+      if (warp == 0 && tq == 0 && r < rows_here) {
+        const float lse_val = (L > 0.f) ? M + __log2f(L) : -INFINITY;
+        if (a.num_splits == 1) {
+          if (a.lse != nullptr) a.lse[orow0 + r] = lse_val;
+        } else {
+          a.part_lse[static_cast<int64_t>(split) * rows_all + orow0 + r] = lse_val;
+        }
+      }
+    }
+    const bool hi = g + 8 < rows_here;
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) {
+      const int j = warp + 4 * k;
+      const int col = j * 8 + 2 * tq;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < kDecodeConsumerWarps; ++w) {
+        const float4 x = co4[(w * (D / 8) + j) * 32 + lane];
+        acc.x = fmaf(wt[0][w], x.x, acc.x);
+        acc.y = fmaf(wt[0][w], x.y, acc.y);
+        acc.z = fmaf(wt[1][w], x.z, acc.z);
+        acc.w = fmaf(wt[1][w], x.w, acc.w);
+      }
+      if (a.num_splits == 1) {
+        T* dst = static_cast<T*>(a.out) + (orow0 + g) * D + col;
+        *reinterpret_cast<uint32_t*>(dst) = pack2<T>(acc.x, acc.y);
+        if (hi) *reinterpret_cast<uint32_t*>(dst + 8 * D) = pack2<T>(acc.z, acc.w);
+      } else {
+        float* dst = a.part_o + (static_cast<int64_t>(split) * rows_all + orow0 + g) * D + col;
+        *reinterpret_cast<float2*>(dst) = make_float2(acc.x, acc.y);
+        if (hi) *reinterpret_cast<float2*>(dst + 8 * D) = make_float2(acc.z, acc.w);
+      }
+    }
+  }
   if (a.counters == nullptr || a.num_splits == 1) return;
 
   // ---- in-launch merge: the last CTA of this row group to arrive merges.
@@ -531,10 +522,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
   }
   named_barrier_sync(1, kDecodeConsumerWarps * 32);
   if (*last_flag == 0) return;
-  const int64_t orow0 = (static_cast<int64_t>(b) * a.Hq + static_cast<int64_t>(hkv) * G) * a.Lq +
-                        static_cast<int64_t>(rg) * kDecodeRows;
-  decode_merge_group<D, T>(a, ring, Cfg::kRingBytes, orow0, min(kDecodeRows, rows_total - rg * kDecodeRows),
-                           static_cast<int64_t>(a.B) * a.Hq * a.Lq);
+  decode_merge_group<D, T>(a, ring, Cfg::kRingBytes, orow0, rows_here, rows_all);
   if (tid == 0) a.counters[blockIdx.y] = 0;  // ready for the next call on this workspace
 }
 

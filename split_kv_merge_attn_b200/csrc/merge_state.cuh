@@ -89,6 +89,13 @@ struct Raw8 {
   }
 };
 
+template <typename T>
+__device__ __forceinline__ void store1(T* p, float x) {
+  if constexpr (std::is_same<T, float>::value) *p = x;
+  else if constexpr (std::is_same<T, __half>::value) *p = __float2half_rn(x);
+  else *p = __float2bfloat16_rn(x);
+}
+
 struct MergeArgs {
   const void* o_parts;
   const float* lse_parts;
@@ -307,6 +314,116 @@ __global__ void __launch_bounds__(256) merge_state_parts_kernel(MergeArgs a) {
     for (int e = 0; e < 8; ++e) v[e] *= inv;
     Vec8<TO>::store(out + row * a.D + c * 8, v);
     if (c == 0 && a.lse != nullptr) a.lse[lrow] = (M == -INFINITY) ? -INFINITY : M + log2f(Wt);
+  }
+}
+
+// Few rows and many parts with D / 8 = VPR in {8, 16} (instantiable for 32):
+// one CTA per row; thread t takes column slice t / LANES and parts t % LANES,
+// t % LANES + LANES, ... (LANES = 256 / VPR consecutive threads of one warp
+// per slice, so the LANES threads of a slice hold every part once).  A thread
+// requests the LSEs and O slices of up to R of its parts at once (one memory
+// round trip per batch), weighs them against its own running max (one exp2
+// per part, one per batch for the rescale), and the slice's threads then agree
+// on the row max and add their weighted sums and weight sums with warp
+// shuffles: no shared memory and no block barrier.  A part of LSE -inf has
+// weight 0 and its O slot is not used.  Launched as a programmatic dependent
+// of the split kernel (griddepcontrol.wait).
+template <typename TI, typename TO, int VPR>
+__global__ void __launch_bounds__(256) merge_parts_shfl_kernel(MergeArgs a) {
+  constexpr int kLanes = 256 / VPR;
+  constexpr int R = 4;  // parts per thread in flight
+  static_assert(kLanes >= 8 && kLanes <= 32, "one slice's part lanes lie inside one warp");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int pl = threadIdx.x % kLanes;
+  const int c = threadIdx.x / kLanes;
+  const int64_t row = blockIdx.x;
+  int64_t lrow = row;
+  if (a.layout_bsh) {
+    const int h = static_cast<int>(row % a.H);
+    const int64_t bs = row / a.H;
+    const int s = static_cast<int>(bs % a.S);
+    const int64_t b = bs / a.S;
+    lrow = (b * a.H + h) * a.S + s;
+  }
+  const TI* __restrict__ base = static_cast<const TI*>(a.o_parts) + row * a.D + c * 8;
+  const float* __restrict__ lb = a.lse_parts + lrow;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float m = -INFINITY, W = 0.f;
+  for (int p0 = pl; p0 < a.P; p0 += R * kLanes) {
+    float L[R];
+    Raw8<TI> x[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {  // every load of the batch is issued before any use
+      const int p = p0 + r * kLanes;
+      L[r] = (p < a.P) ? __ldg(lb + p * a.part_stride_lse) : -INFINITY;
+      if (p < a.P) x[r].load(base + p * a.part_stride_o);
+    }
+    float bm = m;
+#pragma unroll
+    for (int r = 0; r < R; ++r) bm = fmaxf(bm, L[r]);
+    if (bm == -INFINITY) continue;  // no part with weight yet
+    const float sc = (m == -INFINITY) ? 0.f : ex2_approx(m - bm);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] *= sc;
+    W *= sc;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (L[r] == -INFINITY) continue;
+      const float w = ex2_approx(L[r] - bm);
+      float xf[8];
+      x[r].unpack(xf);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, xf[e], acc[e]);
+      W += w;
+    }
+    m = bm;
+  }
+  float M = m;
+#pragma unroll
+  for (int o = kLanes / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float f = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
+  W *= f;
+#pragma unroll
+  for (int o = kLanes / 2; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+  // reduce-scatter of the 8 sums over the slice's threads: at lane distance
+  // 1, 2, 4 each thread keeps one half of what it holds, sends the other half
+  // and adds its partner's (4 + 2 + 1 shuffles); then thread pl holds element
+  // 4 (pl & 1) + 2 (pl >> 1 & 1) + (pl >> 2 & 1) summed over 8 threads, and the
+  // remaining distances (8, 16) add whole values.
+  float h4[4];
+  {
+    const bool up = pl & 1;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float send = up ? acc[e] * f : acc[e + 4] * f;
+      const float keep = up ? acc[e + 4] * f : acc[e] * f;
+      h4[e] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+  }
+  float h2[2];
+  {
+    const bool up = (pl >> 1) & 1;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float send = up ? h4[e] : h4[e + 2];
+      const float keep = up ? h4[e + 2] : h4[e];
+      h2[e] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+  }
+  float v;
+  {
+    const bool up = (pl >> 2) & 1;
+    const float send = up ? h2[0] : h2[1];
+    const float keep = up ? h2[1] : h2[0];
+    v = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+#pragma unroll
+  for (int o = 8; o < kLanes; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (pl < 8) {
+    const int e = 4 * (pl & 1) + 2 * ((pl >> 1) & 1) + ((pl >> 2) & 1);
+    const float inv = (M != -INFINITY && W > 0.f) ? 1.0f / W : 0.f;
+    store1<TO>(static_cast<TO*>(a.out) + row * a.D + c * 8 + e, v * inv);
+    if (c == 0 && pl == 0 && a.lse != nullptr) a.lse[lrow] = (M == -INFINITY) ? -INFINITY : M + __log2f(W);
   }
 }
 

@@ -132,6 +132,10 @@ cudaError_t launch_parts(const MergeArgs& a, unsigned rows, cudaStream_t st, boo
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = dependent ? 1 : 0;
+  // D = 64, 128: the shuffle-reduced kernel; other D (D = 256 measured faster
+  // with the shared-memory reduction in the decode's dependent launch)
+  if (a.D == 64) return cudaLaunchKernelEx(&cfg, merge_parts_shfl_kernel<TI, TO, 8>, a);
+  if (a.D == 128) return cudaLaunchKernelEx(&cfg, merge_parts_shfl_kernel<TI, TO, 16>, a);
   return cudaLaunchKernelEx(&cfg, merge_state_parts_kernel<TI, TO>, a);
 }
 }  // namespace

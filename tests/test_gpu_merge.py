@@ -93,3 +93,29 @@ def test_merge_of_splits_reproduces_full_attention():
                     "HND", out=out, lse=lse)
     check_o(out, o_full, float(d["v"].float().abs().max()))
     check_lse(lse, l_full)
+
+
+@pytest.mark.parametrize("D", [64, 96, 256])
+@pytest.mark.parametrize("P", [8, 40, 200])
+@pytest.mark.parametrize("layout", ["HND", "NHD"])
+def test_merge_few_rows_many_parts(D, P, layout):
+    """The per-row kernels (few rows, P >= 8 parts): several batches of parts
+    per thread at P = 200, empty parts, rows without any part, the
+    slice-by-shuffle variant (D = 64, 256) and the general one (D = 96)."""
+    B, H, S = 1, 3, 5
+    o, l = make_parts(P, (B, H, S, D), (B, H, S), seed=D + P, pdt="fp32", empty_frac=0.3)
+    l[:, 0, 1, 2] = float("-inf")
+    o_ref, l_ref = O.merge(O.to_f64(o), O.to_f64(l))
+    lse = nan_empty((B, H, S), torch.float32)
+    if layout == "HND":
+        out = nan_empty((B, H, S, D), torch.bfloat16)
+        skv.merge_state(o.cuda(), l.cuda(), "HND", out=out, lse=lse)
+        got = out
+    else:
+        out = nan_empty((B, S, H, D), torch.bfloat16)
+        skv.merge_state(o.permute(0, 1, 3, 2, 4).contiguous().cuda(), l.cuda(), "NHD", out=out, lse=lse)
+        got = out.permute(0, 2, 1, 3)
+    torch.cuda.synchronize()
+    check_o(got.contiguous(), o_ref, float(o.abs().max()), tol=8e-3)
+    check_lse(lse, l_ref, tol=1e-4)
+    assert torch.all(lse[0, 1, 2] == float("-inf")) and torch.all(got[0, 1, 2] == 0)
