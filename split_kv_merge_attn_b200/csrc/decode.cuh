@@ -267,20 +267,32 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
 
   // ================= consumer warps
   // Q rows of this group into shared memory (zero rows pad the tile); the
-  // producer's first K/V loads are already in flight meanwhile
+  // producer's first K/V loads are already in flight meanwhile.  Every load of
+  // a thread is issued before its first shared-memory store (one round trip:
+  // the stores could alias the loads' addresses for the compiler, which would
+  // otherwise keep each load behind the previous store).
   {
     constexpr int vpr = D / 8;
-    for (int v = tid; v < kDecodeRows * vpr; v += kDecodeConsumerWarps * 32) {
+    constexpr int kQv = kDecodeRows * vpr / (kDecodeConsumerWarps * 32);  // 16-byte pieces per thread
+    static_assert(kDecodeRows * vpr % (kDecodeConsumerWarps * 32) == 0, "Q pieces divide over the consumers");
+    uint4 qv[kQv];
+#pragma unroll
+    for (int u = 0; u < kQv; ++u) {
+      const int v = tid + kDecodeConsumerWarps * 32 * u;
       const int r = v / vpr, c = v % vpr;
       const int rglob = rg * kDecodeRows + r;
-      uint4 val = make_uint4(0, 0, 0, 0);
+      qv[u] = make_uint4(0, 0, 0, 0);
       if (rglob < rows_total) {
         const int h = hkv * G + rglob / a.Lq;
         const int i = rglob % a.Lq;
         const T* src = static_cast<const T*>(a.q) + ((static_cast<int64_t>(b) * a.Hq + h) * a.Lq + i) * D + c * 8;
-        val = *reinterpret_cast<const uint4*>(src);
+        qv[u] = __ldg(reinterpret_cast<const uint4*>(src));
       }
-      *reinterpret_cast<uint4*>(qs + r * Cfg::kQStride + c * 8) = val;
+    }
+#pragma unroll
+    for (int u = 0; u < kQv; ++u) {
+      const int v = tid + kDecodeConsumerWarps * 32 * u;
+      *reinterpret_cast<uint4*>(qs + (v / vpr) * Cfg::kQStride + (v % vpr) * 8) = qv[u];
     }
   }
   named_barrier_sync(1, kDecodeConsumerWarps * 32);
