@@ -14,14 +14,16 @@
 //              NS shared-memory buffers (128-byte swizzle, no multicast)
 //   warp  9    TMEM allocator and (one elected thread) tcgen05.mma issuer
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [256+D, 256+2D) (D <= 128; at D = 256 O_0 fills [256,512) and S_1, O_1
-// are unused: the MMA order is S_0(j), PV_0(j) with the softmax between).  S_a holds fp32 logits; the softmax writes P_a as
-// packed 16-bit pairs into S_a's first 64 columns, and O_a += P_a V_j reads P_a
-// straight from TMEM (A operand in tensor memory).
+// O_1 [256+D, 256+2D) for D <= 128.  S_a holds fp32 logits; the softmax
+// writes P_a as packed 16-bit pairs into S_a's first 64 columns, and
+// O_a += P_a V_j reads P_a straight from TMEM (A operand in tensor memory).
 //
 // The MMA thread alternates between the tiles (S_0(j), PV_1(j-1), S_1(j),
 // PV_0(j)), so while the softmax warps of one tile exponentiate, the tensor
-// core works on the other tile.
+// core works on the other tile.  At D = 256 (one tile; O_0 fills [256,512))
+// the two S buffers hold the logits of consecutive KV steps instead, in the
+// order S(0) | S(j+1), PV(j): the tensor core computes the next step's
+// logits while the softmax of step j runs.
 //
 // Online softmax in the exp2 domain with a lazily updated running max: the
 // max is only raised (and O_a rescaled in TMEM) when it grows by more than 8
@@ -149,8 +151,8 @@ struct PrefillCfg {
   static constexpr int kQTileBytes = kQKBoxes * kBoxBytes;
   static constexpr int kKTileBytes = kQKBoxes * kBoxBytes;
   static constexpr int kKVTileBytes = kBoxes * kBoxBytes;   // one ring buffer (a V tile; a K tile fits)
-  // D = 256: K_j and V_j only; with one query tile, K_{j+1} loads while the
-  // softmax of step j runs and V_{j+1} while S(j+1) and that softmax run
+  // D = 256: K_j and V_j only; K_{j+1} loads once S(j) is done (while the
+  // softmax of step j runs), V_{j+1} once PV(j) is done (while S(j+2) runs)
   static constexpr int kStages = (D == 64) ? 8 : (D == 256 ? 2 : 5);
   static constexpr int kRingBytes = kStages * kKVTileBytes;
   static constexpr int kOffQ = 0;
@@ -354,12 +356,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           else tma_load_4d(qtile[t] + bx * Cfg::kBoxBytes, &tmQ, q_full, x, h, s, bcoord);
         }
       }
-      int issued = 0;
+      int last_u[Cfg::kStages];  // last load issued into each ring buffer (-1: none)
+#pragma unroll
+      for (int i = 0; i < Cfg::kStages; ++i) last_u[i] = -1;
       bool ok = true;
-      for (int j = 0; j < nkv && ok; ++j) {
+      // Load order: K_0 V_0 K_1 V_1 ... for two query tiles.  With one tile
+      // (D = 256: two ring buffers, K in buffer 0 and V in buffer 1) the MMA
+      // order is S(0) S(1) PV(0) S(2) PV(1) ..., so the buffers free up (and
+      // are refilled) in the order K_0 V_0 K_1 | K_2 V_1 | K_3 V_2 | ...
+      // (n -> u: 3 -> 4, 4 -> 3, 5 -> 6, ...; the one u past the end is skipped)
+      const int n_end = 2 * nkv + (Cfg::kTiles == 1 ? 1 : 0);
+      for (int n = 0; n < n_end && ok; ++n) {
+        int u = n;
+        if (Cfg::kTiles == 1 && n >= 3) u = (n & 1) ? n + 1 : n - 1;
+        if (u >= 2 * nkv) continue;
+        const int j = u >> 1;
         const int s = k_row0 + j * kPfBN;
-        for (int which = 0; which < 2; ++which) {
-          const int u = 2 * j + which;
+        {
+          const int which = u & 1;
           const int buf = u % Cfg::kStages;
           if (u >= Cfg::kStages) {
             if (!mbar_wait(&kv_empty[buf], ((u / Cfg::kStages) & 1) ^ 1, abort_flag, kErrPrefillWait)) {
@@ -378,13 +392,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (hnd) tma_load_4d(dst, m, &kv_full[buf], bx * bxe, s, hkv, bcoord);
             else tma_load_4d(dst, m, &kv_full[buf], bx * bxe, hkv, s, bcoord);
           }
-          issued = u + 1;
+          last_u[buf] = u;
         }
       }
       if (*abort_flag) {
+        // every load issued lands before the CTA's shared memory goes away: a
+        // buffer is refilled only after its previous load was consumed, so only
+        // the last load into each buffer can still be in flight
         mbar_drain(q_full, 0, 20000000ull);
-        for (int u = max(0, issued - Cfg::kStages); u < issued; ++u)
-          mbar_drain(&kv_full[u % Cfg::kStages], (u / Cfg::kStages) & 1, 20000000ull);
+#pragma unroll
+        for (int i = 0; i < Cfg::kStages; ++i)
+          if (last_u[i] >= 0) mbar_drain(&kv_full[i], (last_u[i] / Cfg::kStages) & 1, 20000000ull);
       }
     }
   } else if (warp == 9) {
@@ -464,35 +482,69 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       auto release = [&](int u) { commit(&kv_empty[u % Cfg::kStages]); };
       const bool two = nt == 2;
 
-      bool ok = wait_bar(q_full, 0) && wait_kv(0);
-      if (ok) {
-        issue_s(dq0, s0c, 0);
-        commit(&s_full[0]);
-        if (two) {
-          issue_s(dq1, s1c, 0);
-          commit(&s_full[1]);
+      if constexpr (Cfg::kTiles == 1) {
+        // One query tile (D = 256): S is double-buffered in TMEM columns
+        // [0, 128) and [128, 256), and the order S(0) | S(j+1) PV(j) lets the
+        // tensor core compute the next logits while the softmax of step j
+        // runs.  S(j+1) overwrites the buffer PV(j-1) read P from, issued
+        // before it.  After each PV, o_full[1] tracks its completion: the
+        // softmax of step j+1 waits for it before it rescales O.
+        auto sbuf = [&](int j) { return (j & 1) ? s1c : s0c; };
+        auto wait_p1 = [&](int j, int hf) { return wait_bar(&p_half[2 * (j & 1) + hf], (j >> 1) & 1); };
+        bool ok = wait_bar(q_full, 0) && wait_kv(0);
+        if (ok) {
+          issue_s(dq0, s0c, 0);
+          commit(&s_full[0]);
+          release(0);
         }
-        release(0);
-        ok = wait_kv(1) && issue_pv(0, 1, false, 0);
-        if (ok && nkv == 1) commit(&o_full[0]);
-      }
-      for (int j = 1; j < nkv && ok; ++j) {
-        const int uk = 2 * j, uv = 2 * j + 1;
-        if (!wait_kv(uk)) { ok = false; break; }
-        issue_s(dq0, s0c, uk);
-        commit(&s_full[0]);
-        if (two && !issue_pv(1, uv - 2, j - 1 > 0, j - 1)) { ok = false; break; }
-        release(uv - 2);              // V_{j-1}: both of its PV products are issued
-        if (two) {
-          issue_s(dq1, s1c, uk);
-          commit(&s_full[1]);
+        for (int j = 0; j < nkv && ok; ++j) {
+          if (j + 1 < nkv) {
+            const int uk = 2 * (j + 1);
+            if (!wait_kv(uk)) { ok = false; break; }
+            issue_s(dq0, sbuf(j + 1), uk);
+            commit(&s_full[(j + 1) & 1]);
+            release(uk);
+          }
+          const int uv = 2 * j + 1;
+          if (!wait_kv(uv) || !wait_p1(j, 1)) { ok = false; break; }
+          issue_pv_half(sbuf(j), o0c, uv, j > 0, 1);
+          if (!wait_p1(j, 0)) { ok = false; break; }
+          issue_pv_half(sbuf(j), o0c, uv, j > 0, 0);
+          commit(&o_full[1]);
+          release(uv);
+          if (j == nkv - 1) commit(&o_full[0]);
         }
-        release(uk);                  // K_j: both S products are issued
-        if (!wait_kv(uv)) { ok = false; break; }
-        if (!issue_pv(0, uv, true, j)) { ok = false; break; }
-        if (j == nkv - 1) commit(&o_full[0]);
+      } else {
+        bool ok = wait_bar(q_full, 0) && wait_kv(0);
+        if (ok) {
+          issue_s(dq0, s0c, 0);
+          commit(&s_full[0]);
+          if (two) {
+            issue_s(dq1, s1c, 0);
+            commit(&s_full[1]);
+          }
+          release(0);
+          ok = wait_kv(1) && issue_pv(0, 1, false, 0);
+          if (ok && nkv == 1) commit(&o_full[0]);
+        }
+        for (int j = 1; j < nkv && ok; ++j) {
+          const int uk = 2 * j, uv = 2 * j + 1;
+          if (!wait_kv(uk)) { ok = false; break; }
+          issue_s(dq0, s0c, uk);
+          commit(&s_full[0]);
+          if (two && !issue_pv(1, uv - 2, j - 1 > 0, j - 1)) { ok = false; break; }
+          release(uv - 2);              // V_{j-1}: both of its PV products are issued
+          if (two) {
+            issue_s(dq1, s1c, uk);
+            commit(&s_full[1]);
+          }
+          release(uk);                  // K_j: both S products are issued
+          if (!wait_kv(uv)) { ok = false; break; }
+          if (!issue_pv(0, uv, true, j)) { ok = false; break; }
+          if (j == nkv - 1) commit(&o_full[0]);
+        }
+        if (ok && two && issue_pv(1, 2 * nkv - 1, nkv - 1 > 0, nkv - 1)) commit(&o_full[1]);
       }
-      if (ok && two && issue_pv(1, 2 * nkv - 1, nkv - 1 > 0, nkv - 1)) commit(&o_full[1]);
       // every MMA the elected lane issued has completed before TMEM is released
       commit(drain);
       mbar_drain(drain, 0, 20000000ull);
@@ -504,7 +556,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int row = lg * 32 + lane;    // row inside the tile
     if (t < nt) {
       const uint32_t lane_base = static_cast<uint32_t>(lg * 32) << 16;
-      const uint32_t s_addr = tmem + lane_base + (t == 0 ? Cfg::kSCol0 : Cfg::kSCol1);
+      // one query tile: S of step j in buffer j & 1 (columns [0,128) / [128,256))
+      constexpr bool kSDouble = Cfg::kTiles == 1;
+      const uint32_t s_base = tmem + lane_base + (t == 0 ? Cfg::kSCol0 : Cfg::kSCol1);
       const uint32_t o_addr = tmem + lane_base + (t == 0 ? Cfg::kOCol0 : Cfg::kOCol1);
       const int qi = qblk * Cfg::kRows + t * kPfBM + row;  // row index inside the sequence
       const bool row_valid = qi < len_q;
@@ -569,7 +623,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       float m_run = -INFINITY;  // running max of the (smoothed) log2-domain logits, possibly stale
       float l_run = 0.f;
       for (int j = 0; j < nkv && ok; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, abort_flag, kErrPrefillWait));
+        const int sb = kSDouble ? (j & 1) : t;  // S buffer, and index of its S and P barriers
+        const uint32_t s_addr = kSDouble ? tmem + lane_base + (sb ? Cfg::kSCol1 : Cfg::kSCol0) : s_base;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], kSDouble ? (j >> 1) & 1 : j & 1, abort_flag,
+                                               kErrPrefillWait));
         if (!ok) break;
         tc5::fence_after();
         float sl2 = a.scale_log2;  // log2 units per logit unit of this tile
@@ -613,6 +670,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (j > 0 && __any_sync(0xffffffffu, rescale)) {
           // correction before this tile's P is published: O_t holds the PV
           // products of tiles < j, complete since S_t(j) was issued after them
+          // (one query tile: S(j) is issued before PV(j-1), whose completion
+          // o_full[1] reports; PV(j-2) completed before S(j), so that wait is at
+          // most one phase behind)
+          if constexpr (kSDouble) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&o_full[1], (j - 1) & 1, abort_flag, kErrPrefillWait));
+            if (!ok) break;
+            tc5::fence_after();
+          }
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             float o[32];
@@ -653,7 +718,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc5::ld32(s_addr + 32, *reinterpret_cast<float(*)[32]>(&sh[32]));
         tc5::wait_st();
         tc5::fence_before();
-        mbar_arrive(&p_half[2 * t + 1]);
+        mbar_arrive(&p_half[2 * sb + 1]);
         tc5::wait_ld();
         if constexpr (kI8) s32_to_magic_64(sh);
         if (!full_tile) {
@@ -667,7 +732,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc5::st16(s_addr + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
         tc5::wait_st();
         tc5::fence_before();
-        mbar_arrive(&p_half[2 * t + 0]);
+        mbar_arrive(&p_half[2 * sb + 0]);
         const float2 psa = f2_unpack(ps2[0]), psb = f2_unpack(ps2[1]);
         l_run += (psa.x + psa.y) + (psb.x + psb.y);
       }
