@@ -271,3 +271,29 @@ def test_config5_full_size_sampled():
     a, e = d["chunk_bounds"][c], d["chunk_bounds"][c + 1]
     oc, lc = O.dense(d["q"], d["k"][:, :, a:e], d["v"][:, :, a:e], d["scale"], rows=rows[:40])
     check_lse(torch.stack([l_parts[c, b, h, i] for b, h, i in rows[:40]]), lc)
+
+
+@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_first_half_raises_max_after_second_half_published(D, dtype):
+    """The softmax exponentiates keys [64, 128) of a KV tile first, against the
+    max of those keys; a key in [0, 64) of the same tile that lies far above
+    them (here in the first tile, where O holds only that step's products, and
+    in a later one) makes it wait for the first half's PV products and rescale
+    O before the second half is exponentiated.  Rows alternate between seeing
+    the planted keys as large positive and large negative logits."""
+    B, H, Sq, Sk = 1, 2, 256, 512
+    d = W.dense_case(B, H, H, Sq, Sk, D, seed=21, dtype=dtype)
+    scale = d["scale"]
+    q = d["q"].float()
+    k = d["k"].float()
+    q[:, :, :, 0] = torch.tensor([4.0, -4.0]).repeat(Sq // 2)
+    for pos, logit in [(5, 30.0), (2 * 128 + 40, 70.0)]:
+        k[:, :, pos, :] = 0.0
+        k[:, :, pos, 0] = logit / (4.0 * scale)
+    t = d["q"].dtype
+    d["q"], d["k"] = q.to(t), k.to(t)
+    out, lse = run_dense(d)
+    o_ref, l_ref = O.dense(d["q"], d["k"], d["v"], d["scale"])
+    check_o(out, o_ref, vmax(d["v"]))
+    check_lse(lse, l_ref)
