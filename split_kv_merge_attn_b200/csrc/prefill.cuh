@@ -198,7 +198,8 @@ struct PrefillArgs {
 template <int D, typename T, bool kI8 = false>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const PrefillArgs a) {
   using Cfg = PrefillCfg<D, kI8>;
   static_assert(!kI8 || D == 128, "the int8 path has one 128-byte box per row");
   constexpr int kIsBf16 = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
@@ -740,13 +741,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // ---------------- epilogue: O / l and LSE for this thread's row
       // O rows are staged in an idle K/V ring buffer (this tile's last K tile
       // for tile 0, the last V tile for tile 1: both consumed once o_full
-      // fires) and then written with coalesced 16-byte stores, consecutive
-      // threads covering consecutive bytes of a row.  Chunk c of row r sits
-      // at chunk c ^ (r mod chunks), which keeps the shared-memory accesses of
-      // both phases free of bank conflicts.
-      constexpr int kRowBytes = D * 2;
-      constexpr int kChunks = kRowBytes / 16;
+      // fires) in the layout of the TMA's 128-byte-swizzled 64-column boxes
+      // (16-byte chunk ch of row r in box ch / 8 at position (ch mod 8) ^ (r mod
+      // 8): no shared-memory bank conflicts), then one thread writes the tile
+      // with bulk tensor stores and waits only until they have read shared
+      // memory, so the CTA can retire while the writes drain.  A varlen tile
+      // whose last rows belong to the next sequence is written row by row
+      // instead (coalesced 16-byte stores).
+      constexpr int kChunks = D / 8;  // 16-byte chunks per row
       uint8_t* stg = ring + ((2 * nkv - 2 + t) % Cfg::kStages) * Cfg::kKVTileBytes;
+      auto stg_off = [](int r, int ch) -> uint32_t {
+        return static_cast<uint32_t>(ch >> 3) * Cfg::kBoxBytes + sw128(static_cast<uint32_t>(r), static_cast<uint32_t>(ch & 7));
+      };
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[t], 0, abort_flag, kErrPrefillWait));
       if (ok) {
         tc5::fence_after();
@@ -762,11 +768,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int ch = c * 4 + i;
-            *reinterpret_cast<uint4*>(stg + row * kRowBytes + ((ch ^ (row % kChunks)) * 16)) =
+            *reinterpret_cast<uint4*>(stg + stg_off(row, ch)) =
                 make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
         if (row_valid && a.lse != nullptr) a.lse[lse_idx(qi)] = m_run + __log2f(l_run) + delta;
+        fence_proxy_async_smem();  // the staged rows become visible to the bulk stores
       }
       // every warp of the tile arrives here (an aborted one too, so none waits
       // forever); after an abort the copied rows are garbage and the device
@@ -774,13 +781,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       named_barrier_sync(1 + t, kPfBM);
       if (ok) {
         const int row0 = qblk * Cfg::kRows + t * kPfBM;
+        // dense rows past S_q lie outside the map and are not written
+        if (a.layout != 2 || row0 + kPfBM <= len_q) {
+          if (row == 0) {
+            const int s = q_row0 + t * kPfBM;
+            const int bo = a.layout == 2 ? 0 : chunk * a.B + b;
+#pragma unroll
+            for (int bx = 0; bx < D / 64; ++bx) {
+              if (a.layout == 0) tma_store_4d(&tmO, stg + bx * Cfg::kBoxBytes, bx * 64, s, h, bo);
+              else tma_store_4d(&tmO, stg + bx * Cfg::kBoxBytes, bx * 64, h, s, bo);
+            }
+            bulk_commit_group();
+            bulk_wait_read_all();
+          }
+        } else {
 #pragma unroll 4
-        for (int i = 0; i < kChunks; ++i) {
-          const int idx = i * kPfBM + row;
-          const int r = idx / kChunks, ch = idx % kChunks;
-          if (row0 + r < len_q) {
-            const uint4 val = *reinterpret_cast<const uint4*>(stg + r * kRowBytes + ((ch ^ (r % kChunks)) * 16));
-            *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out_row(row0 + r)) + ch * 16) = val;
+          for (int i = 0; i < kChunks; ++i) {
+            const int idx = i * kPfBM + row;
+            const int r = idx / kChunks, ch = idx % kChunks;
+            if (row0 + r < len_q) {
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + stg_off(r, ch));
+              *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(out_row(row0 + r)) + ch * 16) = val;
+            }
           }
         }
       }

@@ -302,13 +302,13 @@ int make_i8_map(CUtensorMap* m, const void* base, int B, int H, int S) {
 }
 
 template <int D, typename T, bool kI8 = false>
-int launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillArgs& a,
-                     unsigned grid, cudaStream_t st) {
+int launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                     const PrefillArgs& a, unsigned grid, cudaStream_t st) {
   using Cfg = PrefillCfg<D, kI8>;
   auto kern = prefill_kernel<D, T, kI8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kPfThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, a);
+  kern<<<grid, kPfThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
   return counted(cudaGetLastError(), 1);
 }
 
@@ -328,6 +328,11 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
     e = make_qkv_map(&tv, p.v, p.dt, p.layout, Bm, p.Hkv, p.Sk, p.D);
     if (e) return e;
   }
+  // O: the layout of Q, with a multi-chunk call's chunks stacked on the batch axis
+  const int nch_o = (varlen || p.nchunks < 1) ? 1 : p.nchunks;
+  CUtensorMap to;
+  e = make_qkv_map(&to, p.out, p.dt, p.layout, Bm * nch_o, p.Hq, p.Sq > 0 ? p.Sq : 1, p.D);
+  if (e) return e;
   PrefillArgs a;
   a.out = p.out;
   a.lse = p.lse;
@@ -369,13 +374,13 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   if (grid > 0x7fffffff) return cudaErrorInvalidValue;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (p.dt == SKV_BF16) {
-    if (p.D == 64) return launch_prefill_t<64, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
-    if (p.D == 128) return launch_prefill_t<128, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
-    if (p.D == 256) return launch_prefill_t<256, __nv_bfloat16>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+    if (p.D == 64) return launch_prefill_t<64, __nv_bfloat16>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
+    if (p.D == 128) return launch_prefill_t<128, __nv_bfloat16>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
+    if (p.D == 256) return launch_prefill_t<256, __nv_bfloat16>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
   } else {
-    if (p.D == 64) return launch_prefill_t<64, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
-    if (p.D == 128) return launch_prefill_t<128, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
-    if (p.D == 256) return launch_prefill_t<256, __half>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+    if (p.D == 64) return launch_prefill_t<64, __half>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
+    if (p.D == 128) return launch_prefill_t<128, __half>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
+    if (p.D == 256) return launch_prefill_t<256, __half>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
   }
   return cudaErrorInvalidValue;
 }
@@ -444,6 +449,9 @@ int launch_prefill_int8(const Int8PrefillLaunch& p, skv_stream_t stream) {
   if (e) return e;
   e = make_qkv_map(&tv, p.v, p.dt, SKV_HND, p.B, p.Hkv, p.Sk, 128);
   if (e) return e;
+  CUtensorMap to;
+  e = make_qkv_map(&to, p.out, p.dt, SKV_HND, p.B, p.Hq, p.Sq, 128);
+  if (e) return e;
   PrefillArgs a;
   std::memset(&a, 0, sizeof(a));
   a.out = p.out;
@@ -466,8 +474,8 @@ int launch_prefill_int8(const Int8PrefillLaunch& p, skv_stream_t stream) {
   const int64_t grid = static_cast<int64_t>(p.B) * p.Hq * a.nqb;
   if (grid <= 0) return 0;
   if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-  if (p.dt == SKV_BF16) return launch_prefill_t<128, __nv_bfloat16, true>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
-  return launch_prefill_t<128, __half, true>(tq, tk, tv, a, static_cast<unsigned>(grid), st);
+  if (p.dt == SKV_BF16) return launch_prefill_t<128, __nv_bfloat16, true>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
+  return launch_prefill_t<128, __half, true>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
 }
 
 int launch_varlen_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int Hq, int rows_per_cta, int32_t* order,
