@@ -799,6 +799,14 @@ def run_case(args):
         c = W.dense_case(1, 16, 4, 4096, 4096, 256, seed=0)
         q, k, v = c["q"].to(dev), c["k"].to(dev), c["v"].to(dev)
         fn = lambda: skv.attn_fwd_lse(q, k, v, c["scale"])
+    elif case == "prefill_causal":
+        c = W.config5(Sk=4096, n_chunks=1)
+        q, k, v = c["q"].to(dev), c["k"].to(dev), c["v"].to(dev)
+        fn = lambda: skv.attn_fwd_lse(q, k, v, c["scale"], causal=True)
+    elif case == "prefill_int8":
+        c = W.config5(Sk=4096, n_chunks=1)
+        q, k, v = c["q"].to(dev), c["k"].to(dev), c["v"].to(dev)
+        fn = lambda: skv.attn_fwd_lse_int8(q, k, v, c["scale"])
     elif case.startswith("decode_"):
         name = [s for s in DECODE_SHAPES if s[0] == case][0]
         _, Hq, Hkv, D, Lq, Lkv = name
