@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (elect_one()) tc5::commit(smem_u32(bar));
         __syncwarp();
       };
-      // every lane waits; the warp proceeds only on a common verdict
+      // every lane waits; the warp proceeds only on a decision common to all lanes
       auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
         const bool r = __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kErrPrefillWait));
         tc5::fence_after();
