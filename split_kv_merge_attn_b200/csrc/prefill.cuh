@@ -571,13 +571,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (a.kmean != nullptr || a.kpartial != nullptr) {
         const float* mu;
         if (a.kpartial != nullptr) {
-          // mean over this call's KV range from the per-256-key column sums
+          // mean over this call's KV range from the per-256-key column sums.
+          // The column-sum kernel may still be running (this grid can be its
+          // programmatic dependent): wait for its completion first (a no-op
+          // otherwise).  Loads go out sixteen at a time (all of them for a 4096-key
+          // range: one round trip); the sum keeps chunk order.
+          asm volatile("griddepcontrol.wait;" ::: "memory");
           float* mu_s = reinterpret_cast<float*>(smem + Cfg::kOffMu) + t * D;
+          const int nch = (len_k + 255) / 256;
+          const int64_t cstride = static_cast<int64_t>(nseq) * a.Hkv * D;
           for (int d = row; d < D; d += kPfBM) {
-            const int nch = (len_k + 255) / 256;
+            const float* pp = a.kpartial + (static_cast<int64_t>(seq) * a.Hkv + hkv) * D + d;
             float sum = 0.f;
-            for (int c = 0; c < nch; ++c)
-              sum += __ldg(a.kpartial + ((static_cast<int64_t>(c) * nseq + seq) * a.Hkv + hkv) * D + d);
+            int c = 0;
+            for (; c + 16 <= nch; c += 16) {
+              float x[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) x[i] = pp[(c + i) * cstride];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) sum += x[i];
+            }
+            for (; c < nch; ++c) sum += pp[c * cstride];
             mu_s[d] = sum / static_cast<float>(len_k);
           }
           named_barrier_sync(1 + t, kPfBM);

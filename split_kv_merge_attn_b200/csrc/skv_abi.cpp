@@ -283,6 +283,7 @@ skv_status fwd_lse_impl(const void* q, const void* k, const void* v, void* out, 
     if (e) return cuda_status(e);
     if (smooth_k == 1) {
       p.kpartial = partial;   // the prefill kernel sums these into the mean itself
+      p.after_kpartial = max_len > 0 ? 1 : 0;  // the column-sum kernel was the last launch
     } else {
       p.kmean = kmean;
       p.k = kprime;

@@ -74,6 +74,7 @@ struct PrefillLaunch {
   skv_layout layout;
   int nchunks;               // dense: KV chunks (1 = the whole key range)
   const int32_t* kv_bounds;  // host [nchunks + 1] chunk bounds, or null when nchunks == 1
+  int after_kpartial;        // 1: the kernel just launched on the stream is the one writing kpartial
 };
 int launch_prefill(const PrefillLaunch& p, skv_stream_t stream);
 

@@ -303,13 +303,28 @@ int make_i8_map(CUtensorMap* m, const void* base, int B, int H, int S) {
 
 template <int D, typename T, bool kI8 = false>
 int launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
-                     const PrefillArgs& a, unsigned grid, cudaStream_t st) {
+                     const PrefillArgs& a, unsigned grid, cudaStream_t st, bool dependent = false) {
   using Cfg = PrefillCfg<D, kI8>;
   auto kern = prefill_kernel<D, T, kI8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kPfThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
-  return counted(cudaGetLastError(), 1);
+  if (!dependent) {
+    kern<<<grid, kPfThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
+    return counted(cudaGetLastError(), 1);
+  }
+  // programmatic dependent of the K column-sum kernel: CTAs start while it
+  // streams K; only the softmax warps' read of its sums waits for it
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPfThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return counted(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, a), 1);
 }
 
 }  // namespace
@@ -373,17 +388,31 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
   if (grid <= 0) return 0;
   if (grid > 0x7fffffff) return cudaErrorInvalidValue;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool dep = p.after_kpartial != 0 && p.kpartial != nullptr;
   if (p.dt == SKV_BF16) {
-    if (p.D == 64) return launch_prefill_t<64, __nv_bfloat16>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
-    if (p.D == 128) return launch_prefill_t<128, __nv_bfloat16>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
-    if (p.D == 256) return launch_prefill_t<256, __nv_bfloat16>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
+    if (p.D == 64) return launch_prefill_t<64, __nv_bfloat16>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st, dep);
+    if (p.D == 128) return launch_prefill_t<128, __nv_bfloat16>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st, dep);
+    if (p.D == 256) return launch_prefill_t<256, __nv_bfloat16>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st, dep);
   } else {
-    if (p.D == 64) return launch_prefill_t<64, __half>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
-    if (p.D == 128) return launch_prefill_t<128, __half>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
-    if (p.D == 256) return launch_prefill_t<256, __half>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st);
+    if (p.D == 64) return launch_prefill_t<64, __half>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st, dep);
+    if (p.D == 128) return launch_prefill_t<128, __half>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st, dep);
+    if (p.D == 256) return launch_prefill_t<256, __half>(tq, tk, tv, to, a, static_cast<unsigned>(grid), st, dep);
   }
   return cudaErrorInvalidValue;
 }
+
+namespace {
+// K column sums and K' (smooth.cuh): one CTA per unit (256-key chunk, range,
+// kv head) on a 1-D grid
+cudaError_t launch_kmean_partial(const SmoothArgs& a, skv_dtype dt, cudaStream_t st) {
+  const int64_t units = static_cast<int64_t>(a.nchunks) * a.Bseq * a.Hkv;
+  if (units <= 0) return cudaSuccess;
+  if (units > 0x7fffffff) return cudaErrorInvalidValue;
+  if (dt == SKV_BF16) kmean_partial_kernel<__nv_bfloat16><<<static_cast<unsigned>(units), 256, 0, st>>>(a);
+  else kmean_partial_kernel<__half><<<static_cast<unsigned>(units), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+}  // namespace
 
 int launch_prefill_int8(const Int8PrefillLaunch& p, skv_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -407,9 +436,8 @@ int launch_prefill_int8(const Int8PrefillLaunch& p, skv_stream_t stream) {
   sa.kvb[0] = 0;
   sa.kvb[1] = p.Sk;
   {
-    dim3 grid(sa.nchunks, p.B, p.Hkv);
-    if (p.dt == SKV_BF16) kmean_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(sa);
-    else kmean_partial_kernel<__half><<<grid, 256, 0, st>>>(sa);
+    const cudaError_t e = launch_kmean_partial(sa, p.dt, st);
+    if (e != cudaSuccess) return e;
     kmean_finalize_kernel<<<p.B * p.Hkv, 128, 0, st>>>(sa);
     launches += 2;
   }
@@ -541,17 +569,16 @@ int launch_smooth_k(const void* k, void* k_smoothed, float* kmean, float* partia
   a.nchunks = static_cast<int>(ceil_div64(max_len, kSmoothChunk));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (a.nchunks > 0) {
-    dim3 grid(a.nchunks, a.Bseq, Hkv);
-    if (dt == SKV_BF16) kmean_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
-    else kmean_partial_kernel<__half><<<grid, 256, 0, st>>>(a);
+    const cudaError_t e = launch_kmean_partial(a, dt, st);
+    if (e != cudaSuccess) return e;
   }
   // the mean itself is needed here only to materialise K'; otherwise the
   // prefill kernel adds up the per-chunk partial sums of its own KV range
   if (k_smoothed != nullptr) kmean_finalize_kernel<<<a.Bseq * Hkv, D, 0, st>>>(a);
   if (k_smoothed != nullptr && a.nchunks > 0) {
-    dim3 grid(a.nchunks, a.Bseq, Hkv);
-    if (dt == SKV_BF16) ksmooth_write_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
-    else ksmooth_write_kernel<__half><<<grid, 256, 0, st>>>(a);
+    const unsigned units = static_cast<unsigned>(static_cast<int64_t>(a.nchunks) * a.Bseq * Hkv);
+    if (dt == SKV_BF16) ksmooth_write_kernel<__nv_bfloat16><<<units, 256, 0, st>>>(a);
+    else ksmooth_write_kernel<__half><<<units, 256, 0, st>>>(a);
   }
   const int n = (a.nchunks > 0 ? 1 : 0) + (k_smoothed != nullptr ? 1 : 0) +
                 (k_smoothed != nullptr && a.nchunks > 0 ? 1 : 0);

@@ -46,51 +46,93 @@ __device__ __forceinline__ int smooth_len(const SmoothArgs& a, int r) {
   return a.kvb[c + 1] - a.kvb[c];
 }
 
-// grid (nchunks, Bseq, Hkv), 256 threads: (D/8) column vectors x (256/(D/8)) row lanes.
-// Every thread issues its row loads in batches of 16 before summing them (all
-// of its rows of the chunk at D = 128: enough bytes in flight to stream K).
+// row stride (elements) between consecutive keys of one range and kv head
+__device__ __forceinline__ int64_t smooth_row_stride(const SmoothArgs& a) {
+  return a.layout == 0 ? a.D : static_cast<int64_t>(a.Hkv) * a.D;
+}
+
+// A unit is one 256-key chunk c of range r and kv head hkv: block u of the
+// 1-D grid, u = c + nchunks * (r + Bseq * hkv).
+struct KmeanUnit {
+  int c, r, hkv, s0, s1;
+};
+
+__device__ __forceinline__ KmeanUnit kmean_unit(const SmoothArgs& a, int u) {
+  KmeanUnit w;
+  w.c = u % a.nchunks;
+  w.r = (u / a.nchunks) % a.Bseq;
+  w.hkv = u / (a.nchunks * a.Bseq);
+  w.s0 = w.c * kSmoothChunk;
+  w.s1 = min(smooth_len(a, w.r), w.s0 + kSmoothChunk);
+  return w;
+}
+
+// Column sums of one unit per CTA, 256 threads: (D/8) column vectors x
+// (256/(D/8)) row lanes; thread (cv, rl) sums the 16-byte piece cv of rows
+// s0 + rl + i * lanes, loads issued eight at a time.  The unit's base address
+// is computed once and each further row is one pointer step, and 64 registers
+// allow four CTAs per SM: this streams K at the rate of a plain read of it
+// (row addresses recomputed per load made the kernel issue bound at a third of
+// that).  The sums over the row lanes go through warp shuffles (lanes D/8 apart
+// hold the same columns), then the 8 warps' sums through shared memory, added
+// in warp order, so each partial is the same fp32 sum on every run.
+constexpr int kKmeanBatch = 8;
+
 template <typename T>
-__global__ void __launch_bounds__(256) kmean_partial_kernel(SmoothArgs a) {
-  const int c = blockIdx.x, b = blockIdx.y, hkv = blockIdx.z;
-  const int len = smooth_len(a, b);
-  const int vpr = a.D / 8;
-  const int lanes = 256 / vpr;
-  const int cv = threadIdx.x % vpr, rl = threadIdx.x / vpr;
-  const int s0 = c * kSmoothChunk, s1 = min(len, s0 + kSmoothChunk);
+__global__ void __launch_bounds__(256, 4) kmean_partial_kernel(SmoothArgs a) {
+  // a prefill launched as this grid's programmatic dependent may start now:
+  // it reads these sums only after griddepcontrol.wait
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int vpr = a.D / 8, lanes = 256 / vpr;
+  const int cv = tid % vpr, rl = tid / vpr;
+  const int rpt = kSmoothChunk / lanes;  // rows of the unit per thread: 8, 16, 32
+  const KmeanUnit w = kmean_unit(a, blockIdx.x);
+  const int nv = w.s1 - w.s0;            // rows of the unit (none past the range's end)
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  const T* k = static_cast<const T*>(a.k);
-  // rows of this thread: s0 + rl + i * lanes; loads issued in batches of 16
-  constexpr int kBatch = 16;
-  for (int i0 = 0; i0 * lanes < kSmoothChunk; i0 += kBatch) {
-    uint4 u[kBatch];
+  if (nv > 0) {
+    const int64_t rs = smooth_row_stride(a);
+    const int64_t step = lanes * rs;
+    const T* p = static_cast<const T*>(a.k) + smooth_row_off(a, w.r, w.hkv, w.s0) + rl * rs + cv * 8;
+    for (int i0 = 0; i0 < rpt; i0 += kKmeanBatch) {
+      uint4 u[kKmeanBatch];
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const int s = s0 + rl + (i0 + i) * lanes;
-      u[i] = (s < s1) ? __ldg(reinterpret_cast<const uint4*>(k + smooth_row_off(a, b, hkv, s) + cv * 8))
-                      : make_uint4(0, 0, 0, 0);
-    }
+      for (int i = 0; i < kKmeanBatch; ++i)
+        u[i] = (rl + (i0 + i) * lanes < nv) ? __ldg(reinterpret_cast<const uint4*>(p + (i0 + i) * step))
+                                             : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+      for (int i = 0; i < kKmeanBatch; ++i) {
+        const uint32_t x[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = unpack2<T>(w[e]);
-        acc[2 * e] += f.x;
-        acc[2 * e + 1] += f.y;
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack2<T>(x[e]);
+          acc[2 * e] += f.x;
+          acc[2 * e + 1] += f.y;
+        }
       }
     }
   }
-  __shared__ float red[256 * 8];
+  for (int o = vpr; o < 32; o <<= 1)
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[(rl * vpr + cv) * 8 + e] = acc[e];
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+  __shared__ float4 red[8][32][2];  // [warp][column vector][8 floats]
+  if (lane < vpr) {
+    red[warp][lane][0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    red[warp][lane][1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
   __syncthreads();
-  if (rl == 0) {
-    for (int r = 1; r < lanes; ++r)
+  if (tid < vpr) {
+    float4 s0 = red[0][tid][0], s1 = red[0][tid][1];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += red[(r * vpr + cv) * 8 + e];
-    float* dst = a.partial + ((static_cast<int64_t>(c) * a.Bseq + b) * a.Hkv + hkv) * a.D + cv * 8;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) dst[e] = acc[e];
+    for (int wi = 1; wi < 8; ++wi) {
+      const float4 x0 = red[wi][tid][0], x1 = red[wi][tid][1];
+      s0.x += x0.x; s0.y += x0.y; s0.z += x0.z; s0.w += x0.w;
+      s1.x += x1.x; s1.y += x1.y; s1.z += x1.z; s1.w += x1.w;
+    }
+    float4* dst = reinterpret_cast<float4*>(
+        a.partial + ((static_cast<int64_t>(w.c) * a.Bseq + w.r) * a.Hkv + w.hkv) * a.D + tid * 8);
+    dst[0] = s0;
+    dst[1] = s1;
   }
 }
 
@@ -106,23 +148,24 @@ __global__ void kmean_finalize_kernel(SmoothArgs a) {
   a.kmean[static_cast<int64_t>(bh) * a.D + d] = len > 0 ? s / static_cast<float>(len) : 0.f;
 }
 
-// K' = K - mean, rounded to T; grid (nchunks, Bseq, Hkv), 256 threads
+// K' = K - mean, rounded to T; one unit per CTA (as the column sums), 256 threads
 template <typename T>
 __global__ void __launch_bounds__(256) ksmooth_write_kernel(SmoothArgs a) {
-  const int c = blockIdx.x, b = blockIdx.y, hkv = blockIdx.z;
-  const int len = smooth_len(a, b);
+  const KmeanUnit w = kmean_unit(a, blockIdx.x);
   const int vpr = a.D / 8;
   const int lanes = 256 / vpr;
   const int cv = threadIdx.x % vpr, rl = threadIdx.x / vpr;
-  const int s0 = c * kSmoothChunk, s1 = min(len, s0 + kSmoothChunk);
-  const float* mu = a.kmean + (static_cast<int64_t>(b) * a.Hkv + hkv) * a.D + cv * 8;
+  if (w.s1 <= w.s0) return;
+  const float* mu = a.kmean + (static_cast<int64_t>(w.r) * a.Hkv + w.hkv) * a.D + cv * 8;
   float m[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) m[e] = mu[e];
+  const int64_t rs = smooth_row_stride(a);
+  const int64_t base = smooth_row_off(a, w.r, w.hkv, w.s0) + cv * 8;
   const T* k = static_cast<const T*>(a.k);
   T* ko = static_cast<T*>(a.k_out);
-  for (int s = s0 + rl; s < s1; s += lanes) {
-    const int64_t off = smooth_row_off(a, b, hkv, s) + cv * 8;
+  for (int s = w.s0 + rl; s < w.s1; s += lanes) {
+    const int64_t off = base + (s - w.s0) * rs;
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(k + off));
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
     uint32_t o[4];
