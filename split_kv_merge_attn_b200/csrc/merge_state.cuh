@@ -109,23 +109,31 @@ struct MergeArgs {
 };
 
 // Many-row merge (the ring / chunk merge) for D / 8 = VPR slices per row: one
-// thread per 8-element slice; the LSEs and O slices of up to kBatch parts are
+// thread per kSlices adjacent 8-element slices of a row (kSlices * 16 or 32
+// contiguous bytes per part); the LSEs and O slices of up to kBatch parts are
 // all requested before any is used (one memory round trip per batch), then
 // the batch's max is taken first and each part gets one approximate exp2 (no
-// running-max chain inside a batch).  Row arithmetic is 32-bit where the slice
-// count allows it.  A part whose LSE is -inf carries no weight and its O slot
-// (which may hold anything) is not used.
-template <typename TI, typename TO, int VPR, bool kWide>
+// running-max chain inside a batch).  Two slices per thread halve the
+// per-byte share of that weight arithmetic, which every thread of a row
+// repeats, and double the bytes each thread has in flight.  Row arithmetic is
+// 32-bit where the slice count allows it.  A part whose LSE is -inf carries no
+// weight and its O slot (which may hold anything) is not used.
+#ifndef SKV_MERGE_SLICES
+#define SKV_MERGE_SLICES 2
+#endif
+template <typename TI, typename TO, int VPR, bool kWide, int kSlices = SKV_MERGE_SLICES>
 __global__ void __launch_bounds__(256) merge_rows_kernel(MergeArgs a) {
+  static_assert(VPR % kSlices == 0, "slices of a row split evenly over its threads");
   constexpr int kBatch = 4;
+  constexpr int kTpr = VPR / kSlices;  // threads per row
   const TI* __restrict__ op = static_cast<const TI*>(a.o_parts);
   const float* __restrict__ lp = a.lse_parts;
   TO* __restrict__ out = static_cast<TO*>(a.out);
   using Idx = typename std::conditional<kWide, int64_t, int32_t>::type;
   const Idx g = static_cast<Idx>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (g >= a.n_vec) return;
-  const Idx row = g / VPR;
-  const int c = static_cast<int>(g % VPR);
+  if (g >= a.n_vec / kSlices) return;
+  const Idx row = g / kTpr;
+  const int c = static_cast<int>(g % kTpr) * kSlices;  // first slice of this thread
   Idx lrow = row;
   if (a.layout_bsh) {
     const Idx h = row % a.H;
@@ -135,15 +143,21 @@ __global__ void __launch_bounds__(256) merge_rows_kernel(MergeArgs a) {
   const TI* base = op + static_cast<int64_t>(row) * a.D + c * 8;
   const float* lbase = lp + lrow;
   float m = -INFINITY, W = 0.f;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float acc[kSlices][8];
+#pragma unroll
+  for (int k = 0; k < kSlices; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
   for (int p0 = 0; p0 < a.P; p0 += kBatch) {
     float L[kBatch];
-    Raw8<TI> x[kBatch];
+    Raw8<TI> x[kBatch][kSlices];
 #pragma unroll
     for (int r = 0; r < kBatch; ++r) {
       const int p = p0 + r;
       L[r] = (p < a.P) ? __ldg(lbase + p * a.part_stride_lse) : -INFINITY;
-      if (p < a.P) x[r].load(base + p * a.part_stride_o);
+      if (p < a.P)
+#pragma unroll
+        for (int k = 0; k < kSlices; ++k) x[r][k].load(base + p * a.part_stride_o + k * 8);
     }
     float mb = m;
 #pragma unroll
@@ -152,23 +166,31 @@ __global__ void __launch_bounds__(256) merge_rows_kernel(MergeArgs a) {
     const float sc = ex2_approx(m - mb);    // 0 while m is -inf
     W *= sc;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] *= sc;
+    for (int k = 0; k < kSlices; ++k)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[k][e] *= sc;
 #pragma unroll
     for (int r = 0; r < kBatch; ++r) {
       if (L[r] == -INFINITY) continue;      // an empty part: its O slot is not used
       const float w = ex2_approx(L[r] - mb);
-      float xf[8];
-      x[r].unpack(xf);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, xf[e], acc[e]);
+      for (int k = 0; k < kSlices; ++k) {
+        float xf[8];
+        x[r][k].unpack(xf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(w, xf[e], acc[k][e]);
+      }
       W += w;
     }
     m = mb;
   }
   const float inv = (m != -INFINITY && W > 0.f) ? 1.0f / W : 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] *= inv;
-  Vec8<TO>::store(out + static_cast<int64_t>(row) * a.D + c * 8, acc);
+  for (int k = 0; k < kSlices; ++k) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[k][e] *= inv;
+    Vec8<TO>::store(out + static_cast<int64_t>(row) * a.D + (c + k) * 8, acc[k]);
+  }
   if (c == 0 && a.lse != nullptr) a.lse[lrow] = (m == -INFINITY) ? -INFINITY : m + __log2f(W);
 }
 

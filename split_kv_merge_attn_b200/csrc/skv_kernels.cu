@@ -141,11 +141,11 @@ cudaError_t launch_parts(const MergeArgs& a, unsigned rows, cudaStream_t st, boo
 }  // namespace
 
 namespace {
-// Many-row merge with D / 8 = VPR: one thread per slice, one block per 256
-// slices; 32-bit row arithmetic when the slice count fits.
+// Many-row merge with D / 8 = VPR: one thread per SKV_MERGE_SLICES slices,
+// 256 threads a block; 32-bit row arithmetic when the slice count fits.
 template <typename TI, typename TO, int VPR>
 cudaError_t launch_rows(const MergeArgs& a, cudaStream_t st) {
-  const int64_t blocks = (a.n_vec + 255) / 256;
+  const int64_t blocks = (a.n_vec / SKV_MERGE_SLICES + 255) / 256;
   if (a.n_vec < (int64_t(1) << 31) - 256 && static_cast<int64_t>(a.B) * a.H * a.S * a.D < (int64_t(1) << 31))
     merge_rows_kernel<TI, TO, VPR, false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
   else
