@@ -207,6 +207,24 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
   const int hkv = (blockIdx.y / a.row_groups) % a.Hkv;
   const int b = blockIdx.y / (a.row_groups * a.Hkv);
 
+  if (tid == 0) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDecodeConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();  // barriers initialised
+  // This grid is launched as a programmatic dependent of the kernel before it
+  // on the stream, so its CTAs can be resident before that kernel ends: every
+  // thread waits here for that kernel's completion (and its memory) before it
+  // reads an input (kv_len, Q, K, V) or writes anything.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // let a programmatically dependent merge launch be scheduled; it still waits
+  // for this whole grid to finish before it reads the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
   // ---- split bounds (same rule as the host planner)
   int n = a.Lkv;
   if (a.kv_len != nullptr) n = min(max(a.kv_len[b], 0), a.Lkv);
@@ -218,19 +236,6 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
     s1 = min(s0 + C, n);
   }
   const int ntiles = (s1 - s0 + kDecodeKeysPerTile - 1) / kDecodeKeysPerTile;
-
-  if (tid == 0) {
-    for (int s = 0; s < Cfg::kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kDecodeConsumerWarps);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();  // barriers initialised
-  // let a programmatically dependent merge launch be scheduled; it still waits
-  // for this whole grid to finish before it reads the partials
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int64_t row0 = (static_cast<int64_t>(b) * a.Hkv + hkv) * a.Lkv;
 

@@ -262,6 +262,9 @@ __global__ void __launch_bounds__(256) merge_state_kernel(MergeArgs a) {
 template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) merge_state_parts_kernel(MergeArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the next kernel on the stream, if launched as a programmatic dependent
+  // (the next decode's split kernel), may become resident meanwhile
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const TI* __restrict__ op = static_cast<const TI*>(a.o_parts);
   const float* __restrict__ lp = a.lse_parts;
   TO* __restrict__ out = static_cast<TO*>(a.out);
@@ -356,6 +359,9 @@ __global__ void __launch_bounds__(256) merge_parts_shfl_kernel(MergeArgs a) {
   constexpr int R = 4;  // parts per thread in flight
   static_assert(kLanes >= 8 && kLanes <= 32, "one slice's part lanes lie inside one warp");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the next kernel on the stream, if launched as a programmatic dependent
+  // (the next decode's split kernel), may become resident meanwhile
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int pl = threadIdx.x % kLanes;
   const int c = threadIdx.x / kLanes;
   const int64_t row = blockIdx.x;

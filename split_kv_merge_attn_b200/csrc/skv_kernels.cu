@@ -217,8 +217,20 @@ int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeAr
   auto kern = decode_split_kernel<D, T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kDecodeThreads, Cfg::kSmemBytes, st>>>(tk, tv, a);
-  return counted(cudaGetLastError(), 1);
+  // programmatic dependent of the previous kernel on the stream: its CTAs may
+  // become resident (and set up) while that kernel finishes; the kernel waits
+  // (griddepcontrol.wait) before touching memory
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return counted(cudaLaunchKernelEx(&cfg, kern, tk, tv, a), 1);
 }
 }  // namespace
 
