@@ -123,6 +123,10 @@ struct MergeArgs {
 #endif
 template <typename TI, typename TO, int VPR, bool kWide, int kSlices = SKV_MERGE_SLICES>
 __global__ void __launch_bounds__(256) merge_rows_kernel(MergeArgs a) {
+  // launched as a programmatic dependent of the kernel before it (which may
+  // have produced the parts): wait for it before any load
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   static_assert(VPR % kSlices == 0, "slices of a row split evenly over its threads");
   constexpr int kBatch = 4;
   constexpr int kTpr = VPR / kSlices;  // threads per row
@@ -200,6 +204,10 @@ __global__ void __launch_bounds__(256) merge_rows_kernel(MergeArgs a) {
 // for memory once per kBatch parts, not once per part.
 template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) merge_state_kernel(MergeArgs a) {
+  // launched as a programmatic dependent of the kernel before it (which may
+  // have produced the parts): wait for it before any load
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int kBatch = 4;
   const TI* __restrict__ op = static_cast<const TI*>(a.o_parts);
   const float* __restrict__ lp = a.lse_parts;

@@ -336,6 +336,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   __syncthreads();
   tc5::fence_after();
   const uint32_t tmem = *tmem_slot;
+  // a kernel launched as this grid's programmatic dependent (a merge_state of
+  // these partials) may become resident on SMs this grid's last wave leaves
+  // idle; it waits for this grid to finish before it reads anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   uint8_t* qtile[2] = {smem + Cfg::kOffQ, smem + Cfg::kOffQ + Cfg::kQTileBytes};
   uint8_t* ring = smem + Cfg::kOffRing;

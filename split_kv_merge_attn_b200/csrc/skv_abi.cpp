@@ -465,7 +465,7 @@ skv_status decode_impl(const void* q, const void* k, const void* v, void* out, f
   if (splits > 1 && !in_launch_merge) {
     const int64_t rows = static_cast<int64_t>(B) * Hq * Lq;
     e = skv::launch_merge_state(part_o, part_lse, out, lse, splits, 1, 1, static_cast<int>(rows), D, 0, SKV_FP32,
-                                dtype, rows * D, rows, stream, /*dependent=*/true);
+                                dtype, rows * D, rows, stream);
     if (e) return cuda_status(e);
   }
   return SKV_OK;

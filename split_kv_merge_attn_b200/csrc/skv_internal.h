@@ -44,8 +44,7 @@ int sm_count();  // SM count of the current device (cached per device)
 
 int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, float* lse, int P, int B,
                        int H, int S, int D, int layout_bsh, skv_dtype parts_dt, skv_dtype out_dt,
-                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream,
-                       bool dependent = false);
+                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream);
 
 // counters: null = partials only (merge_state merges them); else per-group
 // arrival counters, zero on entry, and the last CTA of each group merges.

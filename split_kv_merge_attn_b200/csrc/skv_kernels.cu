@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "skv_internal.h"
 #include "skv_device.cuh"
@@ -117,26 +118,34 @@ int sm_count() {
 // ------------------------------------------------------------ merge_state
 
 namespace {
-// Launches the per-row merge as a programmatic dependent of the preceding
-// kernel on the stream when `dependent`: its CTAs may become resident during
-// that kernel's tail and start at its completion (griddepcontrol.wait).
-template <typename TI, typename TO>
-cudaError_t launch_parts(const MergeArgs& a, unsigned rows, cudaStream_t st, bool dependent) {
+// Launches `kern` as a programmatic dependent of the kernel before it on the
+// stream: its CTAs may become resident while that kernel finishes.  Every
+// kernel launched this way executes griddepcontrol.wait before it touches
+// memory, so the dependence on the previous kernel's results is kept.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(rows);
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = dependent ? 1 : 0;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// The per-row merge (few rows, many parts): one CTA per row.
+template <typename TI, typename TO>
+cudaError_t launch_parts(const MergeArgs& a, unsigned rows, cudaStream_t st) {
   // D = 64, 128: the shuffle-reduced kernel; other D (D = 256 measured faster
   // with the shared-memory reduction in the decode's dependent launch)
-  if (a.D == 64) return cudaLaunchKernelEx(&cfg, merge_parts_shfl_kernel<TI, TO, 8>, a);
-  if (a.D == 128) return cudaLaunchKernelEx(&cfg, merge_parts_shfl_kernel<TI, TO, 16>, a);
-  return cudaLaunchKernelEx(&cfg, merge_state_parts_kernel<TI, TO>, a);
+  if (a.D == 64) return launch_pdl(merge_parts_shfl_kernel<TI, TO, 8>, dim3(rows), dim3(256), 0, st, a);
+  if (a.D == 128) return launch_pdl(merge_parts_shfl_kernel<TI, TO, 16>, dim3(rows), dim3(256), 0, st, a);
+  return launch_pdl(merge_state_parts_kernel<TI, TO>, dim3(rows), dim3(256), 0, st, a);
 }
 }  // namespace
 
@@ -145,18 +154,16 @@ namespace {
 // 256 threads a block; 32-bit row arithmetic when the slice count fits.
 template <typename TI, typename TO, int VPR>
 cudaError_t launch_rows(const MergeArgs& a, cudaStream_t st) {
-  const int64_t blocks = (a.n_vec / SKV_MERGE_SLICES + 255) / 256;
+  const dim3 blocks(static_cast<unsigned>((a.n_vec / SKV_MERGE_SLICES + 255) / 256));
   if (a.n_vec < (int64_t(1) << 31) - 256 && static_cast<int64_t>(a.B) * a.H * a.S * a.D < (int64_t(1) << 31))
-    merge_rows_kernel<TI, TO, VPR, false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
-  else
-    merge_rows_kernel<TI, TO, VPR, true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
-  return cudaSuccess;
+    return launch_pdl(merge_rows_kernel<TI, TO, VPR, false>, blocks, dim3(256), 0, st, a);
+  return launch_pdl(merge_rows_kernel<TI, TO, VPR, true>, blocks, dim3(256), 0, st, a);
 }
 }  // namespace
 
 int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, float* lse, int P, int B, int H,
                        int S, int D, int layout_bsh, skv_dtype parts_dt, skv_dtype out_dt,
-                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream, bool dependent) {
+                       int64_t part_stride_o, int64_t part_stride_lse, skv_stream_t stream) {
   MergeArgs a;
   a.o_parts = o_parts;
   a.lse_parts = lse_parts;
@@ -186,11 +193,12 @@ int launch_merge_state(const void* o_parts, const float* lse_parts, void* out, f
   cudaError_t le = cudaSuccess;
 #define SKV_MERGE(TI, TO)                                                                   \
   do {                                                                                      \
-    if (per_row) le = launch_parts<TI, TO>(a, static_cast<unsigned>(rows), st, dependent); \
+    if (per_row) le = launch_parts<TI, TO>(a, static_cast<unsigned>(rows), st);            \
     else if (coop && vpr == 8) le = launch_rows<TI, TO, 8>(a, st);                          \
     else if (coop && vpr == 16) le = launch_rows<TI, TO, 16>(a, st);                        \
     else if (coop) le = launch_rows<TI, TO, 32>(a, st);                                     \
-    else merge_state_kernel<TI, TO><<<static_cast<unsigned>(blocks), threads, 0, st>>>(a); \
+    else le = launch_pdl(merge_state_kernel<TI, TO>, dim3(static_cast<unsigned>(blocks)),   \
+                         dim3(threads), 0, st, a);                                          \
   } while (0)
   if (parts_dt == SKV_FP32 && out_dt == SKV_BF16) SKV_MERGE(float, __nv_bfloat16);
   else if (parts_dt == SKV_FP32 && out_dt == SKV_FP16) SKV_MERGE(float, __half);
@@ -217,20 +225,9 @@ int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeAr
   auto kern = decode_split_kernel<D, T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  // programmatic dependent of the previous kernel on the stream: its CTAs may
-  // become resident (and set up) while that kernel finishes; the kernel waits
-  // (griddepcontrol.wait) before touching memory
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(kDecodeThreads);
-  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return counted(cudaLaunchKernelEx(&cfg, kern, tk, tv, a), 1);
+  // programmatic dependent of the previous kernel on the stream (sets up while
+  // that kernel finishes; waits before touching memory)
+  return counted(launch_pdl(kern, grid, dim3(kDecodeThreads), Cfg::kSmemBytes, st, tk, tv, a), 1);
 }
 }  // namespace
 
@@ -414,15 +411,15 @@ int launch_prefill(const PrefillLaunch& p, skv_stream_t stream) {
 }
 
 namespace {
-// K column sums and K' (smooth.cuh): one CTA per unit (256-key chunk, range,
-// kv head) on a 1-D grid
+// K column sums (smooth.cuh): one CTA per unit (256-key chunk, range, kv
+// head) on a 1-D grid, as a programmatic dependent of the kernel before it
 cudaError_t launch_kmean_partial(const SmoothArgs& a, skv_dtype dt, cudaStream_t st) {
   const int64_t units = static_cast<int64_t>(a.nchunks) * a.Bseq * a.Hkv;
   if (units <= 0) return cudaSuccess;
   if (units > 0x7fffffff) return cudaErrorInvalidValue;
-  if (dt == SKV_BF16) kmean_partial_kernel<__nv_bfloat16><<<static_cast<unsigned>(units), 256, 0, st>>>(a);
-  else kmean_partial_kernel<__half><<<static_cast<unsigned>(units), 256, 0, st>>>(a);
-  return cudaGetLastError();
+  const dim3 grid(static_cast<unsigned>(units));
+  if (dt == SKV_BF16) return launch_pdl(kmean_partial_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, a);
+  return launch_pdl(kmean_partial_kernel<__half>, grid, dim3(256), 0, st, a);
 }
 }  // namespace
 

@@ -80,8 +80,12 @@ constexpr int kKmeanBatch = 8;
 
 template <typename T>
 __global__ void __launch_bounds__(256, 4) kmean_partial_kernel(SmoothArgs a) {
-  // a prefill launched as this grid's programmatic dependent may start now:
-  // it reads these sums only after griddepcontrol.wait
+  // launched as a programmatic dependent of the kernel before it (which may
+  // have written K): wait for it before any load.  Then a prefill launched as
+  // this grid's programmatic dependent may start: it reads these sums only
+  // after its own griddepcontrol.wait, and its inputs were complete before
+  // this wait returned.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int vpr = a.D / 8, lanes = 256 / vpr;
