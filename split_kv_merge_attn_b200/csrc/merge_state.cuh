@@ -265,8 +265,9 @@ __global__ void __launch_bounds__(256) merge_state_kernel(MergeArgs a) {
 // running max of its own; the part lanes are then rescaled to the row max and
 // summed through shared memory -- one round trip to memory instead of one per
 // part.  A part of LSE -inf contributes nothing (its O slot is never used in
-// arithmetic).  Launched as a programmatic dependent of the split kernel, it
-// waits for that grid's results with griddepcontrol.wait.
+// arithmetic).  Launched as a programmatic dependent of the kernel before it
+// (the decode's split kernel, or whatever wrote the parts), it waits for that
+// grid's results with griddepcontrol.wait.
 template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) merge_state_parts_kernel(MergeArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(256) merge_state_parts_kernel(MergeArgs a) {
 // on the row max and add their weighted sums and weight sums with warp
 // shuffles: no shared memory and no block barrier.  A part of LSE -inf has
 // weight 0 and its O slot is not used.  Launched as a programmatic dependent
-// of the split kernel (griddepcontrol.wait).
+// of the kernel before it, whose results it waits for (griddepcontrol.wait).
 template <typename TI, typename TO, int VPR>
 __global__ void __launch_bounds__(256) merge_parts_shfl_kernel(MergeArgs a) {
   constexpr int kLanes = 256 / VPR;
