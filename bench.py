@@ -466,6 +466,22 @@ def run_ours(args, rank, world, dist):
         "graph_us": round(us_1, 2), "graph_tflops": round(FLOPS_CFG5 / (us_1 * 1e-6) / 1e12, 1),
         "four_calls_graph_us": round(us_4, 2)})
     del k5c, v5c
+    # workload 1 (B1 H4 S_q 64 S_k 1000 D128): latency bound, microseconds only;
+    # also with K + 0.5 and smooth_k (the repro's third part)
+    c1 = W.config1("rows")
+    q1, k1, v1 = c1["q"].to(dev), c1["k"].to(dev), c1["v"].to(dev)
+    k1s = (c1["k"].float() + 0.5).to(c1["k"].dtype).to(dev)
+    o1 = torch.empty_like(q1)
+    l1 = torch.empty(1, 4, 64, dtype=torch.float32, device=dev)
+    ws1 = torch.empty(skv.attn_fwd_lse_workspace(1, 4, 4, 1000, 128, "bf16", "HND", 1), dtype=torch.uint8,
+                      device=dev)
+    us_1a = time_graph(lambda: skv.attn_fwd_lse(q1, k1, v1, c1["scale"], out=o1, lse=l1), 50)
+    us_1b = time_graph(lambda: skv.attn_fwd_lse(q1, k1s, v1, c1["scale"], smooth_k=1, out=o1, lse=l1,
+                                                workspace=ws1), 50)
+    detail["cfg1_dense_h4_s64_sk1000"] = {"graph_us": round(us_1a, 2), "smooth_k_graph_us": round(us_1b, 2),
+                                          "note": "latency bound (0.131 GFLOP): microseconds only, the replay floor "
+                                                  "included"}
+    del q1, k1, v1, k1s, o1, l1, ws1
     # causal variants: prefill of the first workload-5 chunk with its own queries
     # (Sq = Sk = 4096) and the Lq = 4 decode of workload 2 at Lkv 32768
     k5_0, v5_0 = k5[:, :, b5[0]:b5[1]].contiguous(), v5[:, :, b5[0]:b5[1]].contiguous()  # the first chunk
