@@ -39,6 +39,18 @@
  * asynchronous on `stream` (NULL = the legacy default stream), validate every
  * argument on the host first and launch nothing if validation fails.
  *
+ * Stream order: the results of a call are visible to everything the caller
+ * enqueues after it on the stream, as usual.  To hide launch latency, the
+ * decode's split kernel, the merge_state kernels and the smooth_k column sums
+ * are launched with programmatic stream serialization (their CTAs may start
+ * while the preceding kernel finishes; each waits for that kernel's completion
+ * before it touches memory), and the library's kernels signal their dependents
+ * early (griddepcontrol.launch_dependents).  A kernel the caller itself
+ * launches right after a call WITH the programmatic-serialization attribute
+ * must therefore wait for its predecessor (griddepcontrol.wait /
+ * cudaGridDependencySynchronize) before it reads the call's outputs; kernels
+ * launched without that attribute need nothing.
+ *
  * Element types: bf16 or fp16 for q/k/v/out (q, k, v and out share one type);
  * LSE is always fp32.  Head dimension D in {64, 128, 256} (INT8 prefill: 128).
  * Pointers passed as tensors must be 16-byte aligned.
