@@ -119,9 +119,10 @@ typedef enum { SKV_HND = 0, SKV_NHD = 1, SKV_TND = 2 } skv_layout;
  *      up to scale * sum_d |q_d| |K'_d| * 2^-9, so the LSE of this mode is NOT
  *      held to the 1e-3 log2 accuracy of modes 0 and 1 against the exact
  *      unsmoothed LSE: on randn-like inputs with K offset by 0.5 (the chunked
- *      workload) its error is about 2e-3 log2, and it is accepted within 2e-2.
- *      It equals, to 1e-3, the exact LSE of the logits of the rounded K'
- *      (plus the correction).  Use mode 1 where the LSE accuracy matters.
+ *      workload) its error is about 2e-3 log2, and it grows with |q| |K'|
+ *      (about 2e-2 log2 with query rows scaled up to 4x).  It equals, to 1e-3,
+ *      the exact LSE of the logits of the rounded K' (plus the correction).
+ *      Use mode 1 where the LSE accuracy matters.
  *   Both modes need workspace (see below); for varlen, max_seqlen_k must bound
  *   every key length.
  *

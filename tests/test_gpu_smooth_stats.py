@@ -16,6 +16,7 @@ import torch
 import oracle as O
 import split_kv_merge_attn_b200 as skv
 import workloads as W
+from tests._gpu_helpers import check_lse, check_o, vmax
 
 pytestmark = pytest.mark.gpu
 
@@ -129,11 +130,33 @@ def test_varlen_column_sums_and_mean():
         nbytes = skv.attn_fwd_lse_workspace(len(lens), 6, Hkv, Tk, D, layout="TND", smooth_k=smooth_k)
         assert nbytes == sec["total"]
         ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device="cuda")
-        skv.attn_fwd_lse(q, k, v, d["scale"], layout="TND", cu_seqlens_q=d["cu_seqlens_q"].cuda(),
-                         cu_seqlens_k=d["cu_seqlens_k"].cuda(), max_seqlen_q=d["max_seqlen_q"],
-                         max_seqlen_k=d["max_seqlen_k"], smooth_k=smooth_k, workspace=ws)
+        out, lse = skv.attn_fwd_lse(q, k, v, d["scale"], layout="TND", cu_seqlens_q=d["cu_seqlens_q"].cuda(),
+                                    cu_seqlens_k=d["cu_seqlens_k"].cuda(), max_seqlen_q=d["max_seqlen_q"],
+                                    max_seqlen_k=d["max_seqlen_k"], smooth_k=smooth_k, workspace=ws)
         torch.cuda.synchronize()
         assert skv.device_error() == 0
+        # and the call's own result: the unsmoothed attention of each sequence;
+        # smooth_k = 2 attends over K' = K - mean rounded to 16 bits, so its LSE
+        # is held to the oracle's model of that problem (the same rounding of
+        # each sequence's K', done in float64) instead
+        o_ref, l_ref = O.varlen(d["q"], d["k"], d["v"], d["cu_seqlens_q"], d["cu_seqlens_k"], d["scale"])
+        check_o(out, o_ref, vmax(d["v"]))
+        if smooth_k == 1:
+            check_lse(lse, l_ref)
+        else:
+            q64, k64, v64 = O.to_f64(d["q"]), O.to_f64(d["k"]), O.to_f64(d["v"])
+            cq, ck = d["cu_seqlens_q"].tolist(), d["cu_seqlens_k"].tolist()
+            ref2 = l_ref.copy()
+            for bseq in range(len(lens)):
+                if ck[bseq + 1] == ck[bseq]:
+                    continue  # no keys: LSE -inf in both
+                for hq in range(6):
+                    kk = k64[ck[bseq]:ck[bseq + 1], hq // 2]
+                    kp = torch.from_numpy(kk - kk.mean(0)[None]).float().bfloat16().double().numpy()
+                    _, ref2[hq, cq[bseq]:cq[bseq + 1]], _ = O.smoothed_attention_rows(
+                        q64[cq[bseq]:cq[bseq + 1], hq], kk, v64[ck[bseq]:ck[bseq + 1], hq // 2], d["scale"],
+                        k_smoothed=kp)
+            check_lse(lse, ref2)
         k64 = O.to_f64(d["k"])
         cu = d["cu_seqlens_k"].tolist()
         rows = [[k64[cu[r]:cu[r + 1], h] for h in range(Hkv)] for r in range(len(lens))]
